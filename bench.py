@@ -1,0 +1,459 @@
+"""Benchmark of the VideoMLA latent-KV hot path on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input at
+the Wan-1.3B layer shape: ``videomla_cache_write`` of a 3-frame chunk (4680
+tokens) into slots 18-20 of a 21-slot ring, then ``videomla_attention`` of those
+4680 queries over the 21-frame window (32760 keys), 12 heads.  The ring is
+prefilled (untimed) by the same cache-write kernel.
+
+Metric: TFLOP/s of the step, counted with the algorithmic flops of the absorbed
+form: per (query, key, head) 2 (d_c + d_rope) + 2 d_c = 832,
+plus per (query, head) 2 d_nope d_c (absorption) + 2 d_c d_v (W_uv epilogue),
+plus 2 (d_c + d_rope) d_model per written token.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+N > 1 runs under torchrun, one rank per GPU, each rank an independent replica
+of the workload (no collective on the data path; weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from mla_latent_kv_write_b200 import inputs as I  # noqa: E402
+
+METRIC = "latent-KV MLA attention TFLOP/s and % of B200 bf16 peak, 21-frame window"
+WORKLOAD = I.WORKLOADS["wan_layer"]
+N_SETS = 4  # rotating input sets: 4 x ~60 MB > 126 MB L2
+
+
+def flops_attention(d: I.Dims, B: int, Nq: int, Nk: int) -> float:
+    per_qkh = 2 * (d.d_c + d.d_rope) + 2 * d.d_c
+    per_qh = 2 * d.d_nope * d.d_c + 2 * d.d_c * d.d_v
+    return float(B * d.n_heads * (Nq * Nk * per_qkh + Nq * per_qh))
+
+
+def flops_explicit_equivalent(d: I.Dims, B: int, Nq: int, Nk: int) -> float:
+    # dense MHA on reconstructed keys / values: QK^T over 128 + PV over 128, plus
+    # reconstruction of K_nope and V for every key and head
+    dh = d.d_nope + d.d_rope
+    return float(B * d.n_heads * (Nq * Nk * (2 * dh + 2 * d.d_v) + Nk * 2 * d.d_c * (d.d_nope + d.d_v)))
+
+
+def flops_cache_write(d: I.Dims, B: int, n_tok: int) -> float:
+    return float(2 * B * n_tok * (d.d_c + d.d_rope) * d.d_model)
+
+
+def bytes_cache_write(d: I.Dims, B: int, n_tok: int) -> float:
+    return float(B * n_tok * (2 * d.d_model + 2 * (d.d_c + d.d_rope)))
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            m = json.load(f)
+        return m, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def ncu_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            t = json.load(f)
+        e = t.get(kernel)
+        if not e:
+            return None
+        from mla_latent_kv_write_b200 import build as vb
+        import hashlib
+        h = hashlib.sha256()
+        for s in vb.SOURCES:
+            with open(s, "rb") as fh:
+                h.update(fh.read())
+        if e.get("sources_sha256") != h.hexdigest():
+            return None
+        return e.get("dram_bytes_per_launch")
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4], parts[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[4]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows), "samples": len(loaded), "reasons": reasons}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on a bounded sample of query rows
+# ---------------------------------------------------------------------------
+
+def cpu_oracle_sample(target_s: float = 12.0):
+    from oracle import videomla_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = len(os.sched_getaffinity(0))
+    wl, d = WORKLOAD, WORKLOAD.dims
+    T_f = d.tokens_per_frame
+    seed = I.seed_for(wl.index, 0, 0)
+    w = I.layer_weights(d, seed)
+    q = I.queries(d, 1, wl.n_query, seed + 1)
+    cache = I.latent_cache(d, 1, wl.slots, seed + 2)
+    f = I.to_numpy64
+    args = (f(q["q_nope"]), f(q["q_rope"]), f(w["W_uk"]), f(w["W_uv"]), f(cache), wl.slots, 0, wl.slots,
+            d.grid_h, d.grid_w, d.d_c, d.rope_base, d.pairs)
+    rows = np.arange(16)
+    t0 = time.perf_counter()
+    O.attention_absorbed(*args, query_rows=rows)
+    t_probe = time.perf_counter() - t0
+    n = int(min(wl.n_query, max(16, 16 * target_s / max(t_probe, 1e-3))))
+    rows = np.linspace(0, wl.n_query - 1, n).astype(int)
+    t0 = time.perf_counter()
+    O.attention_absorbed(*args, query_rows=rows)
+    dt = time.perf_counter() - t0
+    fl = flops_attention(d, 1, n, wl.slots * T_f)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": int(cores), "kind": "oracle",
+            "seconds": dt, "query_tokens_per_s": n / dt,
+            "sample": f"attention (absorbed fp64 form) of {n} of {wl.n_query} query rows, all "
+                      f"{d.n_heads} heads, all {wl.slots * T_f} keys; cache write not timed"}
+
+
+def run_reference(args):
+    world, rank, _ = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
+    if rank != 0:
+        return 0
+    vals = []
+    base = None
+    for i in range(args.warmup + args.steps):
+        r = cpu_oracle_sample(target_s=max(2.0, 60.0 / max(1, args.steps + args.warmup)))
+        if i >= args.warmup:
+            vals.append(r["value"])
+            base = r
+    v = statistics.mean(vals)
+    d = WORKLOAD.dims
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": base["seconds"] * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"wan_layer: B=1, 12 heads, d_c=192, d_rope=32, 4680 queries x 32760 keys "
+                               f"(oracle on a bounded row sample per step)"},
+        "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": base["cores"], "kind": "oracle",
+                         "sample": base["sample"]},
+        "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def make_sets(dev, n_sets: int):
+    from mla_latent_kv_write_b200 import videomla as V
+    wl, d = WORKLOAD, WORKLOAD.dims
+    T_f = d.tokens_per_frame
+    sets = []
+    for k in range(n_sets):
+        seed = I.seed_for(wl.index, k, 0)
+        w = {n: t.to(dev) for n, t in I.layer_weights(d, seed).items()}
+        prefill = I.tokens(d, wl.batch, wl.prefill * T_f, seed + 3).to(dev)
+        x = I.tokens(d, wl.batch, wl.chunk * T_f, seed + 4)
+        q = I.queries(d, wl.batch, wl.n_query, seed + 5)
+        cache = torch.zeros(wl.batch, wl.slots * T_f, d.cache_width, dtype=torch.bfloat16, device=dev)
+        V.cache_write(prefill, w["W_dkv"], w["W_kr"], w["gamma"], cache, d, wl.slots, 0)
+        del prefill
+        sets.append({
+            "w": w, "cache": cache, "x": x.to(dev), "q_nope": q["q_nope"].to(dev), "q_rope": q["q_rope"].to(dev),
+            "out": torch.empty(wl.batch, wl.n_query, d.n_heads, d.d_v, dtype=torch.bfloat16, device=dev),
+            "x_host": x.pin_memory(), "q_nope_host": q["q_nope"].pin_memory(),
+            "q_rope_host": q["q_rope"].pin_memory(),
+            "out_host": torch.empty(wl.batch, wl.n_query, d.n_heads, d.d_v, dtype=torch.bfloat16).pin_memory(),
+        })
+    torch.cuda.synchronize()
+    return sets
+
+
+def step(s, ev=None):
+    from mla_latent_kv_write_b200 import videomla as V
+    wl, d = WORKLOAD, WORKLOAD.dims
+    w = s["w"]
+    if ev is not None:
+        ev[0].record()
+    V.cache_write(s["x"], w["W_dkv"], w["W_kr"], w["gamma"], s["cache"], d, wl.slots, wl.prefill)
+    if ev is not None:
+        ev[1].record()
+    V.attention(s["q_nope"], s["q_rope"], w["W_uk"], w["W_uv"], s["cache"], d, wl.slots, 0, wl.slots, out=s["out"])
+    if ev is not None:
+        ev[2].record()
+
+
+def step_e2e(s):
+    """Same step through the public API with host buffers: H2D of the step's
+    inputs (x, q_nope, q_rope) from pinned memory, the two kernels, D2H of out."""
+    for name in ("x", "q_nope", "q_rope"):
+        s[name].copy_(s[name + "_host"], non_blocking=True)
+    step(s)
+    s["out_host"].copy_(s["out"], non_blocking=True)
+
+
+def run_gpu(args):
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    from mla_latent_kv_write_b200 import build as vb
+    from mla_latent_kv_write_b200 import videomla as V
+    if rank == 0:
+        vb.build()
+    barrier(world)
+    V.load_library()
+    wl, d = WORKLOAD, WORKLOAD.dims
+    T_f = d.tokens_per_frame
+    Nk = wl.slots * T_f
+    sets = make_sets(dev, N_SETS)
+    fl_attn = flops_attention(d, wl.batch, wl.n_query, Nk)
+    fl_cw = flops_cache_write(d, wl.batch, wl.n_query)
+    fl_step = fl_attn + fl_cw
+
+    for i in range(args.warmup):
+        step(sets[i % N_SETS])
+    barrier(world)
+    if V.device_status(reset=True) != V.OK:
+        raise RuntimeError("a kernel reported a timed-out device wait during warm-up")
+
+    # ---- timed region: K steps, per-kernel events on the launch stream
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        start.record()
+        for i in range(args.steps):
+            step(sets[i % N_SETS], evs[i])
+        stop.record()
+        barrier(world)
+    ms_local = start.elapsed_time(stop)
+    ms = max_over_ranks(ms_local, world)
+    attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    cw_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    clocks = clk.summary()
+
+    # ---- end to end through host buffers
+    for i in range(max(1, args.warmup)):
+        step_e2e(sets[i % N_SETS])
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        step_e2e(sets[i % N_SETS])
+    e1.record()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    if V.device_status(reset=True) != V.OK:
+        raise RuntimeError("a kernel reported a timed-out device wait")
+
+    # ---- cache_write on a 30-layer stack (494 MB > L2), for its HBM roofline
+    cw_stack = cache_write_stack(dev)
+
+    s0 = sets[0]
+    h2d = sum(s0[n].numel() * s0[n].element_size() for n in ("x", "q_nope", "q_rope"))
+    d2h = s0["out"].numel() * s0["out"].element_size()
+
+    if rank == 0:
+        peaks, peak_src = measured_peaks()
+        sm = clocks.get("sm_mhz")
+        sustained = sm is not None and sm < 1700.0
+        peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+        achieved = fl_attn / (attn_ms * 1e-3) / 1e12
+        value = world * fl_step / (ms * 1e-3 / args.steps) / 1e12
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {
+                "workload": "wan_layer: Wan-1.3B-shaped VideoMLA layer, B=1, 12 heads, d_c=192, d_rope=32, "
+                            "d_nope=96, d_v=128, 30x52 grid, cache_write of 3 frames (4680 tokens) into a "
+                            "21-slot ring + attention of 4680 queries x 32760 keys",
+                "global_batch": wl.batch * world, "query_tokens_per_step": wl.n_query, "keys": Nk,
+                "parallelism": f"replicas x{world} (no data-path collective)",
+                "l2": f"inputs larger than L2: {N_SETS} rotating input sets (~60 MB each)",
+                "flops_per_step": fl_step,
+            },
+            "roofline": {"bound": "tensor", "kernel": "attention_kernel", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak,
+                         "peak_kind": f"{peak_src} bf16 {'sustained' if sustained else 'burst'} "
+                                      f"(median SM clock {sm} MHz)",
+                         "traffic": ncu_traffic("attention_kernel"),
+                         "algorithmic_flops_per_launch": fl_attn},
+            "attention_ms": attn_ms, "cache_write_ms": cw_ms,
+            "query_tokens_per_s": wl.n_query * world / (ms * 1e-3 / args.steps),
+            "explicit_mha_equivalent_tflops": flops_explicit_equivalent(d, wl.batch, wl.n_query, Nk)
+            / (attn_ms * 1e-3) / 1e12,
+            "cache_write_stack": cw_stack,
+            "e2e": {"value": world * fl_step / (e2e_ms * 1e-3 / args.steps) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                    "ms_per_step": e2e_ms / args.steps},
+            "clocks": clocks,
+            "gpu_launches": 2 * args.steps,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_oracle_sample()
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def cache_write_stack(dev, layers: int = 30, reps: int = 3):
+    """cache_write over 30 independent layers (3-frame chunks, 494 MB of x +
+    cache traffic > L2), timed back to back; HBM roofline of that kernel."""
+    from mla_latent_kv_write_b200 import videomla as V
+    wl, d = WORKLOAD, WORKLOAD.dims
+    T_f = d.tokens_per_frame
+    n_tok = wl.chunk * T_f
+    xs, caches, ws = [], [], []
+    for l in range(layers):
+        seed = I.seed_for(4, l, 0)
+        xs.append(I.tokens(d, 1, n_tok, seed).to(dev))
+        ws.append({k: v.to(dev) for k, v in I.layer_weights(d, seed).items()})
+        caches.append(torch.zeros(1, wl.slots * T_f, d.cache_width, dtype=torch.bfloat16, device=dev))
+    def run():
+        for l in range(layers):
+            V.cache_write(xs[l], ws[l]["W_dkv"], ws[l]["W_kr"], ws[l]["gamma"], caches[l], d, wl.slots, wl.prefill)
+    run()
+    torch.cuda.synchronize()
+    evs = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        run()
+        b.record()
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    ms = min(a.elapsed_time(b) for a, b in evs) / layers
+    by = bytes_cache_write(d, 1, n_tok)
+    gbs = by / (ms * 1e-3) / 1e9
+    peaks, src = measured_peaks()
+    return {"layers": layers, "ms_per_layer": ms, "bytes_per_layer": by, "achieved_gbs": gbs,
+            "peak_gbs": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"], "peak_kind": f"{src} HBM copy",
+            "tflops": flops_cache_write(d, 1, n_tok) / (ms * 1e-3) / 1e12}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,157 @@
+/*
+ * videomla.h -- C ABI of the B200 (sm_100a) VideoMLA latent-KV hot path.
+ *
+ * Implements the two inference-time steps of "VideoMLA: Low-Rank Latent KV
+ * Cache for Minute-Scale Autoregressive Video Diffusion" (arXiv 2605.30351):
+ *
+ *   videomla_cache_write  -- project new video tokens into the latent ring
+ *                            cache: c^KV = RMSNorm(W_dkv x) (Sec. 3.1 Eq. 1,
+ *                            App. D.2) and the head-shared, unrotated RoPE key
+ *                            k^R = W_kr x (Sec. 3.2 Eq. 5), FIFO ring of frames
+ *                            (App. D.4).
+ *   videomla_attention    -- multi-head latent attention of a query chunk over
+ *                            the sliding window of that cache, in the absorbed
+ *                            inference form (App. E Eq. 8-12): scores
+ *                            (W_uk,h^T q^nope) . c_j + RoPE3D(q^R) . RoPE3D(k^R_j),
+ *                            divided by sqrt(d_nope + d_rope) (Sec. 3.3 Eq. 7),
+ *                            softmax over the whole window, o_h = W_uv,h sum_j p_j c_j
+ *                            (Eq. 10 without W_O).  Keys and queries get
+ *                            window-local (t, h, w) positions (App. D.5).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers (cudaMalloc / torch CUDA memory)
+ *     on the current device, contiguous row-major, 16-byte aligned.  bf16 means
+ *     IEEE bfloat16 stored as 16-bit words.  The caller owns every buffer and the
+ *     stream; the library allocates no device memory per call and never
+ *     synchronises the stream.  ``stream`` is a cudaStream_t (NULL = legacy
+ *     default stream).
+ *   - Calls are asynchronous: a return of VIDEOMLA_OK means the work was
+ *     validated and enqueued.  A kernel whose bounded device-side wait ran out
+ *     records VIDEOMLA_ETIMEOUT in a device status word, read with
+ *     videomla_device_status().
+ *   - Errors are returned as negative codes (below); no exception crosses the
+ *     ABI and nothing is printed.  videomla_strerror() names a code.
+ *   - Thread safety: calls may be made from several host threads; the only
+ *     shared state is a per-device cache of kernel attributes.
+ */
+#ifndef VIDEOMLA_H
+#define VIDEOMLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VIDEOMLA_OK             0
+#define VIDEOMLA_EINVAL        -1  /* null pointer, bad size, bad window, misaligned  */
+#define VIDEOMLA_EUNSUPPORTED  -2  /* geometry with no compiled kernel instance      */
+#define VIDEOMLA_ECUDA         -3  /* CUDA runtime / driver error at launch          */
+#define VIDEOMLA_ETIMEOUT      -4  /* a bounded device-side wait gave up             */
+#define VIDEOMLA_ENODEVICE     -5  /* no sm_100 device is current                    */
+
+/* Flags of videomla_cache_write. */
+#define VIDEOMLA_CACHE_RAW_LATENT 1u /* cache W_dkv x without the RMSNorm            */
+
+/*
+ * Layer geometry.  d_model = d, n_heads = n_h; d_c = latent width; d_rope =
+ * decoupled RoPE width; d_nope = per-head content width (d_nope + d_rope is the
+ * per-head key width, Sec. 3.2); d_v = per-head value width.  A latent frame is
+ * a grid_h x grid_w patch grid (T_f = grid_h * grid_w tokens, row-major).
+ * pairs_t + pairs_h + pairs_w = d_rope / 2 complex pairs over (t, h, w), laid
+ * out t first, interleaved (2p, 2p+1) (App. D.3: (6, 5, 5) for d_rope = 32).
+ * Pair k of an axis that owns D_a dims of a full (d_nope + d_rope)-dim head
+ * rotates by pos * rope_base^(-2k / D_a) (the highest-frequency bands).
+ * rms_eps is the RMSNorm epsilon.
+ */
+typedef struct videomla_dims {
+    int d_model, n_heads, d_c, d_rope, d_nope, d_v;
+    int grid_h, grid_w;
+    int pairs_t, pairs_h, pairs_w;
+    float rope_base;
+    float rms_eps;
+} videomla_dims;
+
+/*
+ * The attention window over the ring cache (App. D.4-D.5).  The ring holds
+ * ``slots`` frames; logical frame j (0 = oldest valid, 0 <= j < n_valid) lives
+ * in slot (oldest_slot + j) mod slots and gets local temporal coordinate t = j.
+ */
+typedef struct videomla_window {
+    int slots;
+    int oldest_slot;
+    int n_valid;
+} videomla_window;
+
+/*
+ * videomla_cache_write -- write the latent cache rows of a chunk of new tokens.
+ *   x      [batch, n_tok, d_model] bf16: token activations (n_tok a multiple of
+ *          T_f; token t of the chunk belongs to frame t / T_f of the chunk).
+ *   W_dkv  [d_c, d_model]    bf16: KV down-projection (Eq. 1).
+ *   W_kr   [d_rope, d_model] bf16: shared RoPE-key projection (Eq. 5).
+ *   gamma  [d_c] fp32 RMSNorm gain, or NULL for unit gain.
+ *   cache  [batch, slots * T_f, d_c + d_rope] bf16 ring (in/out): frame f of
+ *          the chunk is written to slot (first_slot + f) mod slots; row p of a
+ *          slot holds token p of its frame as [RMSNorm(c) | k^R] (k^R unrotated
+ *          and unnormalised).  Rows of other slots are untouched.
+ *   flags  VIDEOMLA_CACHE_RAW_LATENT to skip the RMSNorm, else 0.
+ * Arithmetic: bf16 inputs, fp32 accumulation and normalisation, bf16 RNE output.
+ * Errors: EINVAL (null, n_tok not a whole number of frames, first_slot out of
+ * range, n_tok / T_f > slots, misaligned), EUNSUPPORTED (d_c + d_rope or d_model
+ * without a kernel instance), ECUDA.
+ */
+int videomla_cache_write(const videomla_dims* dims, const void* x, int batch, int n_tok,
+                         const void* W_dkv, const void* W_kr, const float* gamma,
+                         void* cache, int slots, int first_slot, unsigned flags,
+                         void* stream);
+
+/*
+ * videomla_attention -- latent attention of the newest n_query tokens of the
+ * window over all n_valid * T_f keys of the window (no mask inside it).
+ *   q_nope [batch, n_query, n_heads, d_nope] bf16: per-head content queries (Eq. 4).
+ *   q_rope [batch, n_query, n_heads, d_rope] bf16: per-head UNROTATED q^R (Eq. 6);
+ *          the kernel rotates query i by the position of logical token
+ *          n_valid * T_f - n_query + i of the window.
+ *   W_uk   [n_heads * d_nope, d_c] bf16: key up-projection, head-major row blocks.
+ *   W_uv   [n_heads * d_v, d_c]    bf16: value up-projection, head-major row blocks.
+ *   cache  [batch, slots * T_f, d_c + d_rope] bf16, as written by videomla_cache_write.
+ *   out    [batch, n_query, n_heads, d_v] bf16: per-head outputs W_uv,h (sum_j p_j c_j).
+ *   lse    [batch, n_query, n_heads] fp32 natural-log softmax denominator of the
+ *          scaled scores, or NULL.
+ * Arithmetic: bf16 operands on tcgen05 tensor cores with fp32 accumulation; the
+ * absorbed query q_abs and the probabilities are rounded to bf16 before their
+ * contractions; fp32 online softmax.
+ * Errors: EINVAL (null, window out of range, n_query > n_valid * T_f, misaligned),
+ * EUNSUPPORTED (geometry without a kernel instance), ECUDA.
+ */
+int videomla_attention(const videomla_dims* dims, const void* q_nope, const void* q_rope,
+                       const void* W_uk, const void* W_uv, const void* cache,
+                       const videomla_window* window, int batch, int n_query,
+                       void* out, float* lse, void* stream);
+
+/* Name of an error code (static string, never NULL). */
+const char* videomla_strerror(int code);
+
+/*
+ * Device status word of the current device: VIDEOMLA_OK, or VIDEOMLA_ETIMEOUT if
+ * a kernel gave up a bounded wait since the last reset.  Synchronises the device.
+ * reset != 0 clears the word.  Returns ECUDA if it cannot be read.
+ */
+int videomla_device_status(int reset);
+
+/*
+ * Upper bound, in nanoseconds, of every device-side wait of later launches on
+ * this process (default 2e9).  A wait that runs out makes its kernel record
+ * VIDEOMLA_ETIMEOUT, release its tensor memory and return.  0 restores the
+ * default.  Returns the previous value.
+ */
+uint64_t videomla_set_wait_timeout_ns(uint64_t ns);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int videomla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VIDEOMLA_H */

@@ -1,0 +1,338 @@
+// videomla.cu -- the C ABI (include/videomla.h): argument validation, TMA
+// tensor-map encoding, kernel-instance dispatch and launch.  This is the only
+// translation unit of libvideomla.so; the kernels live in the included headers.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/videomla.h"
+#include "attention.cuh"
+#include "cache_write.cuh"
+#include "ptx.cuh"
+
+namespace {
+
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
+std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
+
+// ----------------------------------------------------------------------------
+// driver entry point for cuTensorMapEncodeTiled (resolved through the runtime,
+// so the library does not link libcuda directly)
+// ----------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+CUtensorMapSwizzle swizzle_of(int bytes) {
+    switch (bytes) {
+        case 32: return CU_TENSOR_MAP_SWIZZLE_32B;
+        case 64: return CU_TENSOR_MAP_SWIZZLE_64B;
+        case 128: return CU_TENSOR_MAP_SWIZZLE_128B;
+        default: return CU_TENSOR_MAP_SWIZZLE_NONE;
+    }
+}
+
+// bf16 tensor map of rank ``rank``: dims/box innermost first, strides in bytes
+// of dims 1..rank-1.
+bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
+              const uint32_t* box, int swizzle_bytes) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t d[5], s[4];
+    cuuint32_t bx[5], es[5];
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        bx[i] = box[i];
+        es[i] = 1;
+        if (i + 1 < rank) s[i] = strides[i];
+    }
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), d, s, bx, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_of(swizzle_bytes), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// sm_100 check, cached per device.
+int check_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return VIDEOMLA_ENODEVICE;
+    static std::atomic<int> ok_mask[64];
+    if (dev >= 0 && dev < 64 && ok_mask[dev].load() == 1) return VIDEOMLA_OK;
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+        return VIDEOMLA_ENODEVICE;
+    if (major != 10) return VIDEOMLA_ENODEVICE;
+    if (dev >= 0 && dev < 64) ok_mask[dev].store(1);
+    return VIDEOMLA_OK;
+}
+
+template <class K>
+int launch_status(K kernel, int smem) {
+    (void)kernel;
+    (void)smem;
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? VIDEOMLA_OK : VIDEOMLA_ECUDA;
+}
+
+bool basic_dims_ok(const videomla_dims* d) {
+    if (!d) return false;
+    if (d->d_model <= 0 || d->n_heads <= 0 || d->d_c <= 0 || d->d_rope <= 0 || d->d_nope <= 0 || d->d_v <= 0)
+        return false;
+    if (d->grid_h <= 0 || d->grid_w <= 0) return false;
+    if (d->d_rope % 2) return false;
+    if (d->pairs_t < 0 || d->pairs_h < 0 || d->pairs_w < 0) return false;
+    if (2 * (d->pairs_t + d->pairs_h + d->pairs_w) != d->d_rope) return false;
+    if (!(d->rope_base > 1.0f) || !(d->rms_eps >= 0.0f)) return false;
+    if ((long long)d->grid_h * d->grid_w > (1 << 24)) return false;
+    return true;
+}
+
+// ----------------------------------------------------------------------------
+// cache_write
+// ----------------------------------------------------------------------------
+template <int DC, int DR>
+int run_cache_write(const videomla_dims* d, const void* x, int B, int n_tok, const void* W_dkv, const void* W_kr,
+                    const float* gamma, void* cache, int slots, int first_slot, unsigned flags, cudaStream_t st) {
+    using C = vmla::CacheWriteCfg<DC, DR>;
+    const int T_f = d->grid_h * d->grid_w;
+    CUtensorMap tx, tw, tr;
+    {
+        const uint64_t dims[3] = {uint64_t(d->d_model), uint64_t(n_tok), uint64_t(B)};
+        const uint64_t str[2] = {uint64_t(d->d_model) * 2, uint64_t(n_tok) * d->d_model * 2};
+        const uint32_t box[3] = {64, 128, 1};
+        if (!make_map(&tx, x, 3, dims, str, box, 128)) return VIDEOMLA_ECUDA;
+    }
+    {
+        const uint64_t dims[2] = {uint64_t(d->d_model), uint64_t(DC)};
+        const uint64_t str[1] = {uint64_t(d->d_model) * 2};
+        const uint32_t box[2] = {64, uint32_t(C::WBOX)};
+        if (!make_map(&tw, W_dkv, 2, dims, str, box, 128)) return VIDEOMLA_ECUDA;
+    }
+    {
+        const uint64_t dims[2] = {uint64_t(d->d_model), uint64_t(DR)};
+        const uint64_t str[1] = {uint64_t(d->d_model) * 2};
+        const uint32_t box[2] = {64, uint32_t(DR)};
+        if (!make_map(&tr, W_kr, 2, dims, str, box, 128)) return VIDEOMLA_ECUDA;
+    }
+    vmla::CacheWriteParams p;
+    p.n_tok = n_tok;
+    p.d_model = d->d_model;
+    p.T_f = T_f;
+    p.slots = slots;
+    p.first_slot = first_slot;
+    p.normalize = (flags & VIDEOMLA_CACHE_RAW_LATENT) ? 0 : 1;
+    p.eps = d->rms_eps;
+    p.gamma = gamma;
+    p.cache = static_cast<__nv_bfloat16*>(cache);
+    p.timeout_ns = g_timeout_ns.load();
+    auto kern = vmla::cache_write_kernel<DC, DR>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+        return VIDEOMLA_ECUDA;
+    dim3 grid((n_tok + C::BM - 1) / C::BM, B);
+    kern<<<grid, C::THREADS, C::SMEM, st>>>(tx, tw, tr, p);
+    return launch_status(kern, C::SMEM);
+}
+
+// ----------------------------------------------------------------------------
+// attention
+// ----------------------------------------------------------------------------
+template <int DC, int DR, int DN, int DV>
+int run_attention(const videomla_dims* d, const void* q_nope, const void* q_rope, const void* W_uk, const void* W_uv,
+                  const void* cache, const videomla_window* win, int B, int Nq, void* out, float* lse,
+                  cudaStream_t st) {
+    using C = vmla::AttnCfg<DC, DR, DN, DV>;
+    const int T_f = d->grid_h * d->grid_w;
+    const int H = d->n_heads;
+    const int rows = win->slots * T_f;
+    vmla::AttnParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.Nq = Nq;
+    p.H = H;
+    p.T_f = T_f;
+    p.grid_w = d->grid_w;
+    p.slots = win->slots;
+    p.oldest = win->oldest_slot;
+    // valid physical rows of the window: one run, or two when the ring wraps
+    if (win->n_valid == win->slots) {
+        p.seg_start[0] = 0;
+        p.seg_len[0] = rows;
+    } else {
+        const int last = win->oldest_slot + win->n_valid;
+        p.seg_start[0] = win->oldest_slot * T_f;
+        p.seg_len[0] = (last <= win->slots ? win->n_valid : win->slots - win->oldest_slot) * T_f;
+        if (last > win->slots) {
+            p.seg_start[1] = 0;
+            p.seg_len[1] = (last - win->slots) * T_f;
+        }
+    }
+    p.n_kt = (p.seg_len[0] + C::BK - 1) / C::BK + (p.seg_len[1] + C::BK - 1) / C::BK;
+    p.q_first = win->n_valid * T_f - Nq;
+    p.n_t = d->pairs_t;
+    p.n_h = d->pairs_h;
+    p.n_w = d->pairs_w;
+    p.tab_h_off = win->slots * p.n_t;
+    p.tab_w_off = p.tab_h_off + d->grid_h * p.n_h;
+    p.tab_total = p.tab_w_off + d->grid_w * p.n_w;
+    if (p.tab_total > vmla::kAttnTableMax) return VIDEOMLA_EUNSUPPORTED;
+    // rope frequencies: an axis owning D_a dims of a full (d_nope + d_rope)-dim
+    // head (h, w: floor(n/3) pairs each, t: the rest) uses base^(-2k / D_a)
+    {
+        const int n_full = (d->d_nope + d->d_rope) / 2;
+        const int full_hw = n_full / 3;
+        const int full_t = n_full - 2 * full_hw;
+        const int cnt[3] = {p.n_t, p.n_h, p.n_w};
+        const int D[3] = {2 * full_t, 2 * full_hw, 2 * full_hw};
+        int pr = 0;
+        for (int a = 0; a < 3; ++a)
+            for (int k = 0; k < cnt[a]; ++k)
+                p.omega[pr++] = float(std::pow(double(d->rope_base), -2.0 * k / double(D[a])));
+    }
+    p.scale_log2 = float(1.4426950408889634 / std::sqrt(double(d->d_nope + d->d_rope)));
+    p.q_rope = static_cast<const __nv_bfloat16*>(q_rope);
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.lse = lse;
+    p.timeout_ns = g_timeout_ns.load();
+
+    CUtensorMap tcc, tcr, tqn, tuk, tuv;
+    {
+        const uint64_t dims[3] = {uint64_t(C::W), uint64_t(rows), uint64_t(B)};
+        const uint64_t str[2] = {uint64_t(C::W) * 2, uint64_t(rows) * C::W * 2};
+        const uint32_t box_c[3] = {64, uint32_t(C::BK), 1};
+        const uint32_t box_r[3] = {uint32_t(DR), uint32_t(C::BK), 1};
+        if (!make_map(&tcc, cache, 3, dims, str, box_c, 128)) return VIDEOMLA_ECUDA;
+        if (!make_map(&tcr, cache, 3, dims, str, box_r, DR * 2)) return VIDEOMLA_ECUDA;
+    }
+    {
+        const uint64_t dims[4] = {uint64_t(DN), uint64_t(H), uint64_t(Nq), uint64_t(B)};
+        const uint64_t str[3] = {uint64_t(DN) * 2, uint64_t(H) * DN * 2, uint64_t(Nq) * H * DN * 2};
+        const uint32_t box[4] = {16, 1, uint32_t(C::BM), 1};
+        if (!make_map(&tqn, q_nope, 4, dims, str, box, 32)) return VIDEOMLA_ECUDA;
+    }
+    {
+        const uint64_t dims[2] = {uint64_t(DC), uint64_t(H) * DN};
+        const uint64_t str[1] = {uint64_t(DC) * 2};
+        const uint32_t box[2] = {64, uint32_t(DN)};
+        if (!make_map(&tuk, W_uk, 2, dims, str, box, 128)) return VIDEOMLA_ECUDA;
+    }
+    {
+        const uint64_t dims[2] = {uint64_t(DC), uint64_t(H) * DV};
+        const uint64_t str[1] = {uint64_t(DC) * 2};
+        const uint32_t box[2] = {64, uint32_t(DV)};
+        if (!make_map(&tuv, W_uv, 2, dims, str, box, 128)) return VIDEOMLA_ECUDA;
+    }
+    auto kern = vmla::attention_kernel<C>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+        return VIDEOMLA_ECUDA;
+    dim3 grid((Nq + C::BM - 1) / C::BM, H, B);
+    kern<<<grid, C::THREADS, C::SMEM, st>>>(tcc, tcr, tqn, tuk, tuv, p);
+    return launch_status(kern, C::SMEM);
+}
+
+}  // namespace
+
+extern "C" {
+
+int videomla_cache_write(const videomla_dims* dims, const void* x, int batch, int n_tok, const void* W_dkv,
+                         const void* W_kr, const float* gamma, void* cache, int slots, int first_slot, unsigned flags,
+                         void* stream) {
+    if (!basic_dims_ok(dims) || !x || !W_dkv || !W_kr || !cache) return VIDEOMLA_EINVAL;
+    if (batch <= 0 || batch > 65535 || n_tok <= 0 || slots <= 0 || first_slot < 0 || first_slot >= slots)
+        return VIDEOMLA_EINVAL;
+    if (flags & ~VIDEOMLA_CACHE_RAW_LATENT) return VIDEOMLA_EINVAL;
+    const long long T_f = (long long)dims->grid_h * dims->grid_w;
+    if (n_tok % T_f != 0 || n_tok / T_f > slots) return VIDEOMLA_EINVAL;
+    if ((long long)slots * T_f > (1ll << 30)) return VIDEOMLA_EINVAL;
+    if (!aligned16(x) || !aligned16(W_dkv) || !aligned16(W_kr) || !aligned16(cache) ||
+        (reinterpret_cast<uintptr_t>(gamma) & 7u))
+        return VIDEOMLA_EINVAL;
+    if (dims->d_model % 64 != 0) return VIDEOMLA_EUNSUPPORTED;
+    if (int rc = check_device()) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int dc = dims->d_c, dr = dims->d_rope;
+#define VMLA_CW(DC_, DR_) \
+    if (dc == DC_ && dr == DR_) return run_cache_write<DC_, DR_>(dims, x, batch, n_tok, W_dkv, W_kr, gamma, cache, slots, first_slot, flags, st);
+    VMLA_CW(192, 32)
+    VMLA_CW(192, 16)
+    VMLA_CW(192, 64)
+    VMLA_CW(96, 32)
+    VMLA_CW(384, 32)
+#undef VMLA_CW
+    return VIDEOMLA_EUNSUPPORTED;
+}
+
+int videomla_attention(const videomla_dims* dims, const void* q_nope, const void* q_rope, const void* W_uk,
+                       const void* W_uv, const void* cache, const videomla_window* window, int batch, int n_query,
+                       void* out, float* lse, void* stream) {
+    if (!basic_dims_ok(dims) || !q_nope || !q_rope || !W_uk || !W_uv || !cache || !window || !out)
+        return VIDEOMLA_EINVAL;
+    const videomla_window w = *window;
+    if (w.slots <= 0 || w.oldest_slot < 0 || w.oldest_slot >= w.slots || w.n_valid < 1 || w.n_valid > w.slots)
+        return VIDEOMLA_EINVAL;
+    const long long T_f = (long long)dims->grid_h * dims->grid_w;
+    if (batch <= 0 || batch > 65535 || n_query <= 0 || n_query > w.n_valid * T_f) return VIDEOMLA_EINVAL;
+    if ((long long)w.slots * T_f > (1ll << 30) || dims->n_heads > 65535) return VIDEOMLA_EINVAL;
+    if (!aligned16(q_nope) || !aligned16(q_rope) || !aligned16(W_uk) || !aligned16(W_uv) || !aligned16(cache) ||
+        !aligned16(out) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+        return VIDEOMLA_EINVAL;
+    if (int rc = check_device()) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int dc = dims->d_c, dr = dims->d_rope, dn = dims->d_nope, dv = dims->d_v;
+#define VMLA_AT(DC_, DR_, DN_, DV_)                        \
+    if (dc == DC_ && dr == DR_ && dn == DN_ && dv == DV_) \
+        return run_attention<DC_, DR_, DN_, DV_>(dims, q_nope, q_rope, W_uk, W_uv, cache, &w, batch, n_query, out, lse, st);
+    VMLA_AT(192, 32, 96, 128)
+    VMLA_AT(192, 16, 112, 128)
+    VMLA_AT(192, 64, 64, 128)
+#undef VMLA_AT
+    return VIDEOMLA_EUNSUPPORTED;
+}
+
+const char* videomla_strerror(int code) {
+    switch (code) {
+        case VIDEOMLA_OK: return "ok";
+        case VIDEOMLA_EINVAL: return "invalid argument";
+        case VIDEOMLA_EUNSUPPORTED: return "unsupported geometry (no compiled kernel instance)";
+        case VIDEOMLA_ECUDA: return "CUDA error";
+        case VIDEOMLA_ETIMEOUT: return "a bounded device-side wait timed out";
+        case VIDEOMLA_ENODEVICE: return "no sm_100 device is current";
+        default: return "unknown error";
+    }
+}
+
+int videomla_device_status(int reset) {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, vmla::g_status, sizeof(int)) != cudaSuccess) return VIDEOMLA_ECUDA;
+    if (reset) {
+        const int z = 0;
+        if (cudaMemcpyToSymbol(vmla::g_status, &z, sizeof(int)) != cudaSuccess) return VIDEOMLA_ECUDA;
+    }
+    return v == 0 ? VIDEOMLA_OK : VIDEOMLA_ETIMEOUT;
+}
+
+uint64_t videomla_set_wait_timeout_ns(uint64_t ns) {
+    return g_timeout_ns.exchange(ns == 0 ? kDefaultTimeoutNs : ns);
+}
+
+int videomla_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,181 @@
+"""ctypes binding of ``libvideomla.so`` (C ABI: ``include/videomla.h``).
+
+Argument marshalling only: tensors are checked for dtype, device, shape and
+contiguity, and their device pointers are passed with the current CUDA stream.
+Every step of the computation runs in the library's sm_100a kernels.  If the
+library is missing or cannot be loaded the calls raise: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+from .inputs import Dims
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LOCK = threading.RLock()
+_LIB: Optional[ctypes.CDLL] = None
+
+OK, EINVAL, EUNSUPPORTED, ECUDA, ETIMEOUT, ENODEVICE = 0, -1, -2, -3, -4, -5
+CACHE_RAW_LATENT = 1
+
+# every symbol the header declares
+EXPORTED = (
+    "videomla_cache_write",
+    "videomla_attention",
+    "videomla_strerror",
+    "videomla_device_status",
+    "videomla_set_wait_timeout_ns",
+    "videomla_version",
+)
+
+
+class VideoMLAError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {strerror(code)} ({code})")
+
+
+class CDims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("d_model", "n_heads", "d_c", "d_rope", "d_nope", "d_v",
+                                            "grid_h", "grid_w", "pairs_t", "pairs_h", "pairs_w")] + [
+        ("rope_base", ctypes.c_float), ("rms_eps", ctypes.c_float)]
+
+
+class CWindow(ctypes.Structure):
+    _fields_ = [("slots", ctypes.c_int), ("oldest_slot", ctypes.c_int), ("n_valid", ctypes.c_int)]
+
+
+def library_path() -> str:
+    return os.environ.get("VIDEOMLA_LIBRARY", os.path.join(_PKG, "libvideomla.so"))
+
+
+def load_library() -> ctypes.CDLL:
+    global _LIB
+    with _LOCK:
+        if _LIB is not None:
+            return _LIB
+        path = library_path()
+        if not os.path.exists(path):
+            raise VideoMLAError(ECUDA, f"{path} is missing; build it with "
+                                       "`python -m mla_latent_kv_write_b200.build`")
+        lib = ctypes.CDLL(path)
+        vp, ci, cu = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint
+        lib.videomla_cache_write.argtypes = [ctypes.POINTER(CDims), vp, ci, ci, vp, vp, vp, vp, ci, ci, cu, vp]
+        lib.videomla_cache_write.restype = ci
+        lib.videomla_attention.argtypes = [ctypes.POINTER(CDims), vp, vp, vp, vp, vp, ctypes.POINTER(CWindow),
+                                           ci, ci, vp, vp, vp]
+        lib.videomla_attention.restype = ci
+        lib.videomla_strerror.argtypes = [ci]
+        lib.videomla_strerror.restype = ctypes.c_char_p
+        lib.videomla_device_status.argtypes = [ci]
+        lib.videomla_device_status.restype = ci
+        lib.videomla_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+        lib.videomla_set_wait_timeout_ns.restype = ctypes.c_uint64
+        lib.videomla_version.argtypes = []
+        lib.videomla_version.restype = ci
+        _LIB = lib
+        return lib
+
+
+_NAMES = {OK: "ok", EINVAL: "invalid argument", EUNSUPPORTED: "unsupported geometry",
+          ECUDA: "CUDA error", ETIMEOUT: "device-side wait timed out", ENODEVICE: "no sm_100 device"}
+
+
+def strerror(code: int) -> str:
+    """Name of a status code (host-side table; the library's
+    ``videomla_strerror`` gives the same names)."""
+    return _NAMES.get(code, f"unknown error {code}")
+
+
+def c_dims(d: Dims) -> CDims:
+    return CDims(d.d_model, d.n_heads, d.d_c, d.d_rope, d.d_nope, d.d_v, d.grid_h, d.grid_w,
+                 d.pairs[0], d.pairs[1], d.pairs[2], d.rope_base, d.rms_eps)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _check(t: torch.Tensor, name: str, dtype: torch.dtype, shape=None, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def cache_write(x: torch.Tensor, W_dkv: torch.Tensor, W_kr: torch.Tensor, gamma: Optional[torch.Tensor],
+                cache: torch.Tensor, dims: Dims, slots: int, first_slot: int, raw_latent: bool = False,
+                stream=None) -> torch.Tensor:
+    """Write the latent cache rows of the tokens ``x`` [B, n_tok, d_model] into
+    ``cache`` [B, slots*T_f, d_c + d_rope] (in place; returns ``cache``)."""
+    lib = load_library()
+    B, n_tok = x.shape[0], x.shape[1]
+    dev = x.device
+    _check(x, "x", torch.bfloat16, (B, n_tok, dims.d_model))
+    _check(W_dkv, "W_dkv", torch.bfloat16, (dims.d_c, dims.d_model), dev)
+    _check(W_kr, "W_kr", torch.bfloat16, (dims.d_rope, dims.d_model), dev)
+    if gamma is not None:
+        _check(gamma, "gamma", torch.float32, (dims.d_c,), dev)
+    _check(cache, "cache", torch.bfloat16, (B, slots * dims.tokens_per_frame, dims.cache_width), dev)
+    cd = c_dims(dims)
+    rc = lib.videomla_cache_write(ctypes.byref(cd), _ptr(x), B, n_tok, _ptr(W_dkv), _ptr(W_kr), _ptr(gamma),
+                                  _ptr(cache), slots, first_slot, CACHE_RAW_LATENT if raw_latent else 0,
+                                  _stream(stream))
+    if rc != OK:
+        raise VideoMLAError(rc, "videomla_cache_write")
+    return cache
+
+
+def attention(q_nope: torch.Tensor, q_rope: torch.Tensor, W_uk: torch.Tensor, W_uv: torch.Tensor,
+              cache: torch.Tensor, dims: Dims, slots: int, oldest: int, n_valid: int,
+              out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+              want_lse: bool = False, stream=None):
+    """Latent attention of the queries over the window; returns ``out``
+    [B, Nq, H, d_v] (and ``lse`` [B, Nq, H] if requested or given)."""
+    lib = load_library()
+    B, Nq, H = q_nope.shape[0], q_nope.shape[1], dims.n_heads
+    dev = q_nope.device
+    _check(q_nope, "q_nope", torch.bfloat16, (B, Nq, H, dims.d_nope))
+    _check(q_rope, "q_rope", torch.bfloat16, (B, Nq, H, dims.d_rope), dev)
+    _check(W_uk, "W_uk", torch.bfloat16, (H * dims.d_nope, dims.d_c), dev)
+    _check(W_uv, "W_uv", torch.bfloat16, (H * dims.d_v, dims.d_c), dev)
+    _check(cache, "cache", torch.bfloat16, (B, slots * dims.tokens_per_frame, dims.cache_width), dev)
+    if out is None:
+        out = torch.empty(B, Nq, H, dims.d_v, dtype=torch.bfloat16, device=dev)
+    _check(out, "out", torch.bfloat16, (B, Nq, H, dims.d_v), dev)
+    if lse is None and want_lse:
+        lse = torch.empty(B, Nq, H, dtype=torch.float32, device=dev)
+    if lse is not None:
+        _check(lse, "lse", torch.float32, (B, Nq, H), dev)
+    cd = c_dims(dims)
+    win = CWindow(slots, oldest, n_valid)
+    rc = lib.videomla_attention(ctypes.byref(cd), _ptr(q_nope), _ptr(q_rope), _ptr(W_uk), _ptr(W_uv),
+                                _ptr(cache), ctypes.byref(win), B, Nq, _ptr(out), _ptr(lse), _stream(stream))
+    if rc != OK:
+        raise VideoMLAError(rc, "videomla_attention")
+    return (out, lse) if lse is not None else out
+
+
+def device_status(reset: bool = False) -> int:
+    return load_library().videomla_device_status(1 if reset else 0)
+
+
+def set_wait_timeout_ns(ns: int) -> int:
+    return load_library().videomla_set_wait_timeout_ns(ns)

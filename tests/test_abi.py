@@ -1,0 +1,130 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point that include/videomla.h declares, names its error codes, and
+rejects invalid arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mla_latent_kv_write_b200 import build as vbuild
+from mla_latent_kv_write_b200 import inputs as I
+from mla_latent_kv_write_b200 import videomla as V
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(videomla_\w+)\s*\(", text))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    vbuild.build()
+    return V.load_library()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    declared = declared_symbols()
+    assert declared, "no declarations found"
+    assert declared == set(V.EXPORTED)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_strerror_and_version(lib):
+    assert lib.videomla_version() >= 100
+    for code in (V.OK, V.EINVAL, V.EUNSUPPORTED, V.ECUDA, V.ETIMEOUT, V.ENODEVICE):
+        assert lib.videomla_strerror(code)
+    assert b"unknown" in lib.videomla_strerror(12345)
+
+
+def _dims(**kw):
+    return V.c_dims(I.Dims(**kw) if kw else I.WAN)
+
+
+P = ctypes.c_void_p(0x10000)  # a fake, 16-byte aligned device address: never dereferenced
+
+
+def test_cache_write_rejects_bad_arguments(lib):
+    d = _dims()
+    f = lib.videomla_cache_write
+    T_f = 1560
+    ok_args = [ctypes.byref(d), P, 1, 3 * T_f, P, P, None, P, 21, 18, 0, None]
+    def call(**over):
+        a = list(ok_args)
+        for i, v in over.items():
+            a[int(i[1:])] = v
+        return f(*a)
+    assert call(a1=None) == V.EINVAL                      # x null
+    assert call(a4=None) == V.EINVAL                      # W_dkv null
+    assert call(a7=None) == V.EINVAL                      # cache null
+    assert call(a3=T_f + 1) == V.EINVAL                   # not a whole number of frames
+    assert call(a3=22 * T_f) == V.EINVAL                  # more frames than slots
+    assert call(a9=21) == V.EINVAL                        # first_slot out of range
+    assert call(a9=-1) == V.EINVAL
+    assert call(a2=0) == V.EINVAL                         # batch
+    assert call(a10=8) == V.EINVAL                        # unknown flag
+    assert call(a1=ctypes.c_void_p(0x10008)) == V.EINVAL  # misaligned
+    assert f(None, *ok_args[1:]) == V.EINVAL              # dims null
+    bad = _dims(); bad.pairs_t = 7                         # pairs do not cover d_rope
+    assert f(ctypes.byref(bad), *ok_args[1:]) == V.EINVAL
+    odd = _dims(); odd.d_model = 1000                      # d_model not a multiple of 64
+    assert f(ctypes.byref(odd), *ok_args[1:]) == V.EUNSUPPORTED
+
+
+def test_attention_rejects_bad_arguments(lib):
+    d = _dims()
+    f = lib.videomla_attention
+    win = V.CWindow(21, 0, 21)
+    ok_args = [ctypes.byref(d), P, P, P, P, P, ctypes.byref(win), 1, 4680, P, None, None]
+    def call(**over):
+        a = list(ok_args)
+        for i, v in over.items():
+            a[int(i[1:])] = v
+        return f(*a)
+    for i in (1, 2, 3, 4, 5, 9):
+        assert call(**{f"a{i}": None}) == V.EINVAL
+    assert call(a6=None) == V.EINVAL
+    for w in ((0, 0, 1), (21, 21, 1), (21, -1, 1), (21, 0, 0), (21, 0, 22)):
+        bad = V.CWindow(*w)
+        assert call(a6=ctypes.byref(bad)) == V.EINVAL
+    assert call(a8=21 * 1560 + 1) == V.EINVAL             # more queries than window tokens
+    assert call(a8=0) == V.EINVAL
+    assert call(a10=ctypes.c_void_p(0x10002)) == V.EINVAL  # misaligned lse
+
+
+def test_valid_call_without_device_reports_no_device(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    d = _dims()
+    win = V.CWindow(21, 0, 21)
+    rc = lib.videomla_attention(ctypes.byref(d), P, P, P, P, P, ctypes.byref(win), 1, 4680, P, None, None)
+    assert rc == V.ENODEVICE
+    rc = lib.videomla_cache_write(ctypes.byref(d), P, 1, 4680, P, P, None, P, 21, 18, 0, None)
+    assert rc == V.ENODEVICE
+
+
+def test_unsupported_geometry_is_reported(lib):
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("the geometry check follows the device check")
+    d = _dims(); d.d_c = 160
+    win = V.CWindow(21, 0, 21)
+    P2 = ctypes.c_void_p(0x10000)
+    assert lib.videomla_attention(ctypes.byref(d), P2, P2, P2, P2, P2, ctypes.byref(win), 1, 16, P2, None,
+                                  None) == V.EUNSUPPORTED
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    monkeypatch.setenv("VIDEOMLA_LIBRARY", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(V, "_LIB", None)
+    with pytest.raises(V.VideoMLAError):
+        V.load_library()

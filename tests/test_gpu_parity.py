@@ -1,0 +1,189 @@
+"""GPU parity of the sm_100a kernels against the fp64 oracle, through the C ABI.
+
+Sizes: the tiny 6 x 8 grid (several key tiles, ragged tails, two-run ring
+windows, ragged query counts, batch 2) checked element by element, and the
+Wan-1.3B-shaped workloads at full size checked on sampled query rows (rows are
+independent, so each sampled row is exact) with every head and every key.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from mla_latent_kv_write_b200 import inputs as I
+from mla_latent_kv_write_b200 import videomla as V
+from tests.common import (check_attention, check_cache, check_lse, f64, oracle_attention, oracle_cache,
+                          sample_rows, to_bf16)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _dev(d):
+    return {k: v.to(DEV) for k, v in d.items()}
+
+
+def _attention_case(dims, B, slots, oldest, n_valid, Nq, seed, rows=None, rope_scale=1.0):
+    w = I.layer_weights(dims, seed)
+    q = I.queries(dims, B, Nq, seed + 1)
+    cache = I.latent_cache(dims, B, slots, seed + 2, rope_scale=rope_scale)
+    wd, qd = _dev(w), _dev(q)
+    out, lse = V.attention(qd["q_nope"], qd["q_rope"], wd["W_uk"], wd["W_uv"], cache.to(DEV), dims,
+                           slots, oldest, n_valid, want_lse=True)
+    torch.cuda.synchronize()
+    assert V.device_status(reset=True) == V.OK
+    ref_out, ref_lse = oracle_attention(dims, q, w, cache, slots, oldest, n_valid, rows)
+    got_out, got_lse = f64(out.cpu()), f64(lse.cpu())
+    if rows is not None:
+        got_out, got_lse = got_out[:, rows], got_lse[:, rows]
+    what = f"attention {dims.d_c}/{dims.d_rope} B={B} slots={slots} oldest={oldest} n_valid={n_valid} Nq={Nq}"
+    err = got_out - ref_out
+    print(f"\n{what}: rms rel {np.linalg.norm(err) / np.linalg.norm(ref_out):.2e} "
+          f"max abs {np.max(np.abs(err)):.2e} lse {np.max(np.abs(got_lse - ref_lse)):.2e}")
+    check_attention(got_out, ref_out, what)
+    check_lse(got_lse, ref_lse, "lse")
+
+
+# ---------------------------------------------------------------------------
+# attention
+# ---------------------------------------------------------------------------
+
+def test_attention_tiny_config():
+    # 6 x 8 grid, 1 query frame vs a 3-frame window (144 keys: one full and one ragged tile)
+    _attention_case(I.TINY, B=1, slots=3, oldest=0, n_valid=3, Nq=48, seed=11)
+
+
+@pytest.mark.parametrize("slots,oldest,n_valid,Nq,B", [
+    (7, 4, 5, 100, 2),    # ring wraps: two runs of rows, ragged tiles in both, ragged query tile
+    (7, 0, 7, 336, 1),    # full window, 3 query tiles with a ragged one
+    (5, 2, 1, 48, 1),     # a single valid frame
+    (6, 5, 6, 129, 2),    # full window starting at the last slot, 2 query tiles (second has 1 row)
+    (3, 1, 2, 96, 1),     # window not yet full, contiguous run that does not start at slot 0
+])
+def test_attention_ragged_windows(slots, oldest, n_valid, Nq, B):
+    _attention_case(I.TINY, B=B, slots=slots, oldest=oldest, n_valid=n_valid, Nq=Nq, seed=13 + slots + oldest)
+
+
+def test_attention_wan_layer_sampled_rows():
+    # 4680 queries x 32760 keys, 12 heads, every output computed on the GPU
+    dims = I.WAN
+    rows = sample_rows(4680, 96, seed=5)
+    _attention_case(dims, B=1, slots=21, oldest=0, n_valid=21, Nq=4680, seed=1001, rows=rows)
+
+
+def test_attention_wan_wrapped_window_sampled_rows():
+    dims = I.WAN
+    rows = sample_rows(1560, 48, seed=6)
+    _attention_case(dims, B=1, slots=21, oldest=13, n_valid=21, Nq=1560, seed=1002, rows=rows)
+
+
+@pytest.mark.parametrize("d_c,d_rope", [(192, 16), (192, 64)])
+def test_attention_sweep_points(d_c, d_rope):
+    dims = dataclasses.replace(I.sweep_dims(d_c, d_rope), grid_h=6, grid_w=8)
+    _attention_case(dims, B=2, slots=5, oldest=3, n_valid=4, Nq=150, seed=4000 + d_rope)
+
+
+def test_attention_peaky_scores():
+    # rope keys scaled x8 make scores peaky (std ~ 4): online-softmax rescaling is exercised
+    _attention_case(I.TINY, B=1, slots=7, oldest=2, n_valid=7, Nq=200, seed=17, rope_scale=8.0)
+
+
+def test_attention_long_window_peaky_tokens():
+    """Minute-scale workload: batch 2, 63-frame ring (98280 keys), 4680 queries;
+    1% of the tokens of x scaled x8 before the (oracle) cache write, so their
+    unnormalised rope keys make scores peaky.  Sampled rows, all heads / keys."""
+    wl = I.WORKLOADS["long"]
+    dims = wl.dims
+    T_f = dims.tokens_per_frame
+    seed = I.seed_for(wl.index)
+    w = I.layer_weights(dims, seed)
+    x = I.tokens(dims, wl.batch, wl.slots * T_f, seed + 3, wl.peaky_fraction, wl.peaky_scale)
+    cache = to_bf16(oracle_cache(dims, x, w, wl.slots, 0))
+    del x
+    q = I.queries(dims, wl.batch, wl.n_query, seed + 5)
+    wd, qd = _dev(w), _dev(q)
+    out = V.attention(qd["q_nope"], qd["q_rope"], wd["W_uk"], wd["W_uv"], cache.to(DEV), dims, wl.slots, 0, wl.slots)
+    torch.cuda.synchronize()
+    assert V.device_status(reset=True) == V.OK
+    rows = sample_rows(wl.n_query, 24, seed=7)
+    ref, _ = oracle_attention(dims, q, w, cache, wl.slots, 0, wl.slots, rows)
+    rms_rel, max_abs = check_attention(f64(out.cpu())[:, rows], ref, "long window")
+    print(f"\nlong window: rms rel {rms_rel:.2e} max abs {max_abs:.2e}")
+
+
+# ---------------------------------------------------------------------------
+# cache_write
+# ---------------------------------------------------------------------------
+
+def _cache_write_case(dims, B, frames, slots, first_slot, seed, raw=False):
+    w = I.layer_weights(dims, seed, random_gamma=True)
+    x = I.tokens(dims, B, frames * dims.tokens_per_frame, seed + 1)
+    sentinel = I.latent_cache(dims, B, slots, seed + 2)
+    cache = sentinel.clone().to(DEV)
+    wd = _dev(w)
+    V.cache_write(x.to(DEV), wd["W_dkv"], wd["W_kr"], wd["gamma"], cache, dims, slots, first_slot, raw_latent=raw)
+    torch.cuda.synchronize()
+    assert V.device_status(reset=True) == V.OK
+    ref = oracle_cache(dims, x, w, slots, first_slot, base=f64(sentinel), normalize=not raw)
+    got = f64(cache.cpu())
+    T_f = dims.tokens_per_frame
+    written = np.zeros(slots, dtype=bool)
+    for f in range(frames):
+        written[(first_slot + f) % slots] = True
+    for s in range(slots):
+        sl = slice(s * T_f, (s + 1) * T_f)
+        if written[s]:
+            check_cache(got[:, sl], ref[:, sl], dims.d_c, f"slot {s}")
+        else:
+            assert np.array_equal(got[:, sl], f64(sentinel)[:, sl]), f"slot {s} was modified"
+
+
+def test_cache_write_tiny_wraps_ring():
+    _cache_write_case(I.TINY, B=2, frames=2, slots=3, first_slot=2, seed=21)
+
+
+def test_cache_write_wan_chunk():
+    # 3 frames = 4680 tokens: 36 full token tiles and a ragged one, into slots 18-20
+    _cache_write_case(I.WAN, B=1, frames=3, slots=21, first_slot=18, seed=22)
+
+
+def test_cache_write_raw_latent():
+    _cache_write_case(I.TINY, B=1, frames=3, slots=4, first_slot=1, seed=23, raw=True)
+
+
+@pytest.mark.parametrize("d_c,d_rope", I.SWEEP_POINTS)
+def test_cache_write_sweep_points(d_c, d_rope):
+    dims = dataclasses.replace(I.sweep_dims(d_c, d_rope), grid_h=6, grid_w=8)
+    _cache_write_case(dims, B=1, frames=3, slots=5, first_slot=4, seed=24 + d_c + d_rope)
+
+
+# ---------------------------------------------------------------------------
+# the whole path: rolling ring of 40 frame steps
+# ---------------------------------------------------------------------------
+
+def test_rolling_chain_40_steps():
+    """Frame-by-frame rollout on a 21-slot ring of 30 x 52 frames: each step writes
+    one frame (GPU cache_write) then attends 1560 queries over the window (GPU
+    attention); the oracle runs the same chain with its own fp64 cache rounded
+    to bf16.  Outputs are compared on sampled rows at every step."""
+    wl = I.WORKLOADS["rolling"]
+    dims = wl.dims
+    T_f = dims.tokens_per_frame
+    w = I.layer_weights(dims, I.seed_for(wl.index))
+    wd = _dev(w)
+    cache = torch.zeros(1, wl.slots * T_f, dims.cache_width, dtype=torch.bfloat16, device=DEV)
+    ref_cache = np.zeros((1, wl.slots * T_f, dims.cache_width))
+    for step in range(wl.steps):
+        rw = I.rolling_window(step, wl.slots)
+        x = I.tokens(dims, 1, T_f, I.seed_for(wl.index, 0, 100 + step))
+        q = I.queries(dims, 1, T_f, I.seed_for(wl.index, 0, 200 + step))
+        V.cache_write(x.to(DEV), wd["W_dkv"], wd["W_kr"], wd["gamma"], cache, dims, wl.slots, rw["write_slot"])
+        qd = _dev(q)
+        out = V.attention(qd["q_nope"], qd["q_rope"], wd["W_uk"], wd["W_uv"], cache, dims, wl.slots,
+                          rw["oldest"], rw["n_valid"])
+        oracle_cache(dims, x, w, wl.slots, rw["write_slot"], base=ref_cache)
+        rows = sample_rows(T_f, 12, seed=step)
+        ref_out, _ = oracle_attention(dims, q, w, to_bf16(ref_cache), wl.slots, rw["oldest"], rw["n_valid"], rows)
+        check_attention(f64(out.cpu())[:, rows], ref_out, f"step {step}")
+    assert V.device_status(reset=True) == V.OK
