@@ -393,7 +393,7 @@ def run_gpu(args):
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                     "ms_per_step": e2e_ms / args.steps},
             "clocks": clocks,
-            "gpu_launches": 2 * args.steps,
+            "gpu_launches": 3 * args.steps,  # cache_write, window pre-pass, attention
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_oracle_sample()

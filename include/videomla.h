@@ -107,6 +107,13 @@ int videomla_cache_write(const videomla_dims* dims, const void* x, int batch, in
                          void* stream);
 
 /*
+ * Bytes of the workspace that videomla_attention needs for this window and
+ * batch: the window's rotated RoPE keys, batch * slots * T_f * d_rope fp16
+ * values.  0 for invalid arguments.
+ */
+size_t videomla_attention_workspace_size(const videomla_dims* dims, const videomla_window* window, int batch);
+
+/*
  * videomla_attention -- latent attention of the newest n_query tokens of the
  * window over all n_valid * T_f keys of the window (no mask inside it).
  *   q_nope [batch, n_query, n_heads, d_nope] bf16: per-head content queries (Eq. 4).
@@ -119,16 +126,24 @@ int videomla_cache_write(const videomla_dims* dims, const void* x, int batch, in
  *   out    [batch, n_query, n_heads, d_v] bf16: per-head outputs W_uv,h (sum_j p_j c_j).
  *   lse    [batch, n_query, n_heads] fp32 natural-log softmax denominator of the
  *          scaled scores, or NULL.
- * Arithmetic: bf16 operands on tcgen05 tensor cores with fp32 accumulation; the
- * absorbed query q_abs and the probabilities are rounded to bf16 before their
- * contractions; fp32 online softmax.
- * Errors: EINVAL (null, window out of range, n_query > n_valid * T_f, misaligned),
- * EUNSUPPORTED (geometry without a kernel instance), ECUDA.
+ *   workspace  device scratch of at least videomla_attention_workspace_size()
+ *          bytes, 16-byte aligned, owned by the caller; its contents on entry do
+ *          not matter and are overwritten (the window's rotated RoPE keys,
+ *          App. D.5: rotation applied when the active window is formed).  Calls
+ *          that run concurrently need distinct workspaces.
+ * Two launches on ``stream``: the window pre-pass, then the attention kernel.
+ * Arithmetic: tcgen05 tensor cores with fp32 accumulation; the latent part of
+ * the scores uses bf16 operands (q_abs rounded to bf16), the RoPE part fp16
+ * operands (rotated q^R and k^R), the probabilities are rounded to bf16 before
+ * the sum over latents; fp32 online softmax.
+ * Errors: EINVAL (null, window out of range, n_query > n_valid * T_f, small
+ * workspace, misaligned), EUNSUPPORTED (geometry without a kernel instance), ECUDA.
  */
 int videomla_attention(const videomla_dims* dims, const void* q_nope, const void* q_rope,
                        const void* W_uk, const void* W_uv, const void* cache,
                        const videomla_window* window, int batch, int n_query,
-                       void* out, float* lse, void* stream);
+                       void* out, float* lse, void* workspace, size_t workspace_bytes,
+                       void* stream);
 
 /* Name of an error code (static string, never NULL). */
 const char* videomla_strerror(int code);

@@ -8,12 +8,14 @@
 // over every key of the ring window (App. D.4), with keys and queries rotated
 // by their window-local (t, h, w) positions (App. D.5).
 //
-// One CTA per (128-query tile, head, batch element); 256 threads:
-//   warp 0     TMA producer: q_nope / W_uk (prologue), key tiles (128 keys x
-//              [c | k^R]) into a 3-stage ring, W_uv (epilogue)
+// A pre-pass (rope_window_kernel) forms the active window once per call: every
+// valid cached k^R is rotated by its window-local position into an fp16
+// workspace.  Then one CTA per (128-query tile, head, batch element), 192 threads:
+//   warp 0     TMA producer: q_nope / W_uk (prologue), key tiles (128 keys:
+//              latent from the cache, rotated rope key from the workspace) into
+//              a 4-stage ring, W_uv (epilogue)
 //   warp 1     tcgen05.mma issuer and tensor-memory owner
-//   warps 2-3  RoPE transform: rotate each landed k^R tile in shared memory
-//   warps 4-7  softmax: q_abs -> bf16 Q in TMEM, q^R rotation, fp32 online
+//   warps 2-5  softmax: q_abs -> bf16 Q in TMEM, q^R rotation, fp32 online
 //              softmax (row max / sum reduced across the 4 threads of a row
 //              with warp shuffles), P -> TMEM, O rescale, normalisation,
 //              W_uv epilogue and the output stores
@@ -29,16 +31,13 @@
 
 namespace vmla {
 
-constexpr int kAttnTableMax = 2048;  // float2 (cos, sin) entries of the rope tables
-
 struct AttnParams {
     int Nq, H;
     int T_f, grid_w, slots, oldest;
     int seg_start[2], seg_len[2];  // valid physical key rows: up to two contiguous runs
     int n_kt;                      // key tiles
     int q_first;                   // logical window index of query 0
-    int n_t, n_h, n_w;             // rope pairs per axis
-    int tab_h_off, tab_w_off, tab_total;
+    int n_t, n_h;                  // rope pairs of the t and h axes (w takes the rest)
     float omega[32];               // rope frequency of each pair
     float scale_log2;              // log2(e) / sqrt(d_nope + d_rope)
     const __nv_bfloat16* q_rope;   // [B, Nq, H, DR]
@@ -47,16 +46,28 @@ struct AttnParams {
     uint64_t timeout_ns;
 };
 
+// TMA descriptors of one launch.  The key tensors get one map per valid run of
+// ring rows whose row extent ends at the end of the run, so a ragged last tile
+// reads zeros (never rows of slots outside the window).
+struct AttnMaps {
+    CUtensorMap cc[2];  // cache latent part, per run: (d_c + d_rope, run rows, B), box (64, BK, 1), 128B swizzle
+    CUtensorMap kr[2];  // rotated rope keys (fp16), per run: (d_rope, run rows, B), box (d_rope, BK, 1)
+    CUtensorMap qn;     // q_nope (d_nope, H, Nq, B), box (16, 1, BM, 1), 32B swizzle
+    CUtensorMap wuk;    // W_uk (d_c, H * d_nope), box (64, d_nope), 128B swizzle
+    CUtensorMap wuv;    // W_uv (d_c, H * d_v), box (64, d_v), 128B swizzle
+};
+
 template <int DC_, int DR_, int DN_, int DV_>
 struct AttnCfg {
     static constexpr int DC = DC_, DR = DR_, DN = DN_, DV = DV_;
     static constexpr int W = DC + DR;  // cached scalars per token
-    static constexpr int BM = 128, BK = 128, NS = 3;
+    static constexpr int BM = 128, BK = 128;
     static constexpr int C_ATOMS = DC / 64;
     static constexpr int C_ATOM = BK * 128;           // one 64-column block of the key tile
-    static constexpr int R_ROWB = DR * 2;             // bytes of k^R per key
+    static constexpr int R_ROWB = DR * 2;             // bytes of rotated k^R per key (fp16)
     static constexpr uint32_t R_SW = DR == 16 ? SW32 : DR == 32 ? SW64 : SW128;
     static constexpr int STAGE = C_ATOMS * C_ATOM + BK * R_ROWB;
+    static constexpr int NS = (4 * STAGE + 2048 <= 232448) ? 4 : 3;  // pipeline stages
     static constexpr int O_COL = 0, S_COL = DC, P_COL = DC + BK, Q_COL = DC + BK + BK / 2;
     static constexpr int TMEM_END = Q_COL + W / 2;
     static constexpr int QN_CHUNKS = DN / 16;
@@ -64,8 +75,8 @@ struct AttnCfg {
     static constexpr int WUK_ATOM = DN * 128, WUK_BYTES = C_ATOMS * WUK_ATOM;
     static constexpr int WUV_ATOM = DV * 128, WUV_BYTES = C_ATOMS * WUV_ATOM;
     static constexpr int OLAT_ATOM = BM * 128;
-    static constexpr int SMEM = NS * STAGE + kAttnTableMax * 8 + 512 + 1024;
-    static constexpr int THREADS = 256;
+    static constexpr int SMEM = NS * STAGE + 1024 + 1024;
+    static constexpr int THREADS = 192;
     static_assert(DC % 64 == 0 && DC <= 256, "latent width");
     static_assert(DR == 16 || DR == 32 || DR == 64, "rope width");
     static_assert(DN % 16 == 0 && DV % 32 == 0 && DV <= 256, "head widths");
@@ -75,47 +86,75 @@ struct AttnCfg {
 };
 
 struct AttnBarriers {
-    uint64_t full[4], empty[4], rot[4];
+    uint64_t full[4], empty[4];
     uint64_t q_full, qabs_done, q_ready, s_full, s_free, p_full, pv_done, olat_ready, out_full, drain;
     uint32_t tmem_base;
     AbortState ab;
 };
 
+// Key tile j -> (run, first row inside the run, valid rows).
 template <int BK>
-__device__ __forceinline__ void key_tile(const AttnParams& p, int j, int& start, int& valid) {
+__device__ __forceinline__ void key_tile(const AttnParams& p, int j, int& run, int& row, int& valid) {
     const int t0 = (p.seg_len[0] + BK - 1) / BK;
-    const int s = j < t0 ? 0 : 1;
-    const int jj = j < t0 ? j : j - t0;
-    start = p.seg_start[s] + jj * BK;
-    valid = min(BK, p.seg_len[s] - jj * BK);
+    run = j < t0 ? 0 : 1;
+    row = (j < t0 ? j : j - t0) * BK;
+    valid = min(BK, p.seg_len[run] - row);
 }
 
-// (cos, sin) of pair ``pr`` at grid position (t, hh, ww).
-__device__ __forceinline__ float2 rope_cs(const float2* tab, const AttnParams& p, int pr, int t, int hh, int ww) {
-    if (pr < p.n_t) return tab[t * p.n_t + pr];
-    if (pr < p.n_t + p.n_h) return tab[p.tab_h_off + hh * p.n_h + (pr - p.n_t)];
-    return tab[p.tab_w_off + ww * p.n_w + (pr - p.n_t - p.n_h)];
+// Rotate the pair (x, y) by theta: (x cos - y sin, x sin + y cos), packed as
+// fp16x2.  The RoPE part of the score contraction runs as its own fp16 x fp16
+// MMAs, whose 11-bit significand keeps the rounding of the rotated vectors 8x
+// below bf16 (values are O(10), far inside the fp16 range).
+__device__ __forceinline__ uint32_t rotate_pair(uint32_t v_bf16x2, float theta) {
+    float sn, cs;
+    sincosf(theta, &sn, &cs);
+    const float x = bf16_lo(v_bf16x2), y = bf16_hi(v_bf16x2);
+    return pack_f16(x * cs - y * sn, x * sn + y * cs);
 }
 
-// Rotate one packed bf16 pair (x in the low half) by (cos, sin); the rotated
-// pair is packed as fp16: the RoPE part of the score contraction runs as its own
-// fp16 x fp16 MMAs, whose 11-bit significand keeps the rounding of the rotated
-// vectors 8x below bf16 (values are O(10), far inside the fp16 range).
-__device__ __forceinline__ uint32_t rotate_pair(uint32_t v, float2 cs) {
-    const float x = bf16_lo(v), y = bf16_hi(v);
-    return pack_f16(x * cs.x - y * cs.y, x * cs.y + y * cs.x);
+// Angle of rope pair ``pr`` at window-local position (t, hh, ww).
+__device__ __forceinline__ float rope_theta(const AttnParams& p, int pr, int t, int hh, int ww) {
+    const int pos = pr < p.n_t ? t : (pr < p.n_t + p.n_h ? hh : ww);
+    return float(pos) * p.omega[pr];
+}
+
+// Forming the active window (App. D.5): rotate every valid cached k^R of the
+// window by its window-local (t, h, w) position, once per call, into the fp16
+// workspace [B, slots * T_f, DR] (same row indexing as the cache).  One thread
+// per (batch, valid row, 4 pairs).
+template <int DC, int DR>
+__global__ void __launch_bounds__(256) rope_window_kernel(const __nv_bfloat16* __restrict__ cache,
+                                                          __half* __restrict__ krot, const AttnParams p, int B) {
+    constexpr int W = DC + DR, CH = DR / 8;
+    const int rows_valid = p.seg_len[0] + p.seg_len[1];
+    const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= (long long)B * rows_valid * CH) return;
+    const int ch = int(gid % CH);
+    const long long t2 = gid / CH;
+    const int vr = int(t2 % rows_valid);
+    const int b = int(t2 / rows_valid);
+    const int R = vr < p.seg_len[0] ? p.seg_start[0] + vr : p.seg_start[1] + (vr - p.seg_len[0]);
+    const int slot = R / p.T_f;
+    const int pp = R - slot * p.T_f;
+    int t = slot - p.oldest;
+    if (t < 0) t += p.slots;
+    const int hh = pp / p.grid_w, ww = pp - (pp / p.grid_w) * p.grid_w;
+    const size_t row = size_t(b) * p.slots * p.T_f + R;
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(cache + row * W + DC) + ch);
+    uint4 o;
+    o.x = rotate_pair(v.x, rope_theta(p, 4 * ch + 0, t, hh, ww));
+    o.y = rotate_pair(v.y, rope_theta(p, 4 * ch + 1, t, hh, ww));
+    o.z = rotate_pair(v.z, rope_theta(p, 4 * ch + 2, t, hh, ww));
+    o.w = rotate_pair(v.w, rope_theta(p, 4 * ch + 3, t, hh, ww));
+    reinterpret_cast<uint4*>(krot + row * DR)[ch] = o;
 }
 
 template <class C>
-__global__ void __launch_bounds__(256, 1)
-    attention_kernel(const __grid_constant__ CUtensorMap tm_cc, const __grid_constant__ CUtensorMap tm_cr,
-                     const __grid_constant__ CUtensorMap tm_qn, const __grid_constant__ CUtensorMap tm_wuk,
-                     const __grid_constant__ CUtensorMap tm_wuv, const AttnParams p) {
+__global__ void __launch_bounds__(192, 1) attention_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     constexpr int DC = C::DC, DR = C::DR, DN = C::DN, DV = C::DV, BM = C::BM, BK = C::BK, NS = C::NS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float2* tab = reinterpret_cast<float2*>(smem + NS * C::STAGE);
-    AttnBarriers* bar = reinterpret_cast<AttnBarriers*>(smem + NS * C::STAGE + kAttnTableMax * 8);
+    AttnBarriers* bar = reinterpret_cast<AttnBarriers*>(smem + NS * C::STAGE);
     AbortState* ab = &bar->ab;
     auto stage = [&](int s) { return smem + s * C::STAGE; };
 
@@ -129,7 +168,6 @@ __global__ void __launch_bounds__(256, 1)
         for (int s = 0; s < NS; ++s) {
             mbar_init(&bar->full[s], 1);
             mbar_init(&bar->empty[s], 1);
-            mbar_init(&bar->rot[s], 2);
         }
         mbar_init(&bar->q_full, 1);
         mbar_init(&bar->qabs_done, 1);
@@ -148,25 +186,6 @@ __global__ void __launch_bounds__(256, 1)
         tmem_alloc(&bar->tmem_base, 512);
         tmem_relinquish();
     }
-    // rope tables: [t][n_t] then [h][n_h] then [w][n_w] of (cos, sin)(pos * omega)
-    for (int e = threadIdx.x; e < p.tab_total; e += blockDim.x) {
-        int pos, pr;
-        if (e < p.tab_h_off) {
-            pos = e / p.n_t;
-            pr = e - pos * p.n_t;
-        } else if (e < p.tab_w_off) {
-            const int e2 = e - p.tab_h_off;
-            pos = e2 / p.n_h;
-            pr = p.n_t + (e2 - pos * p.n_h);
-        } else {
-            const int e2 = e - p.tab_w_off;
-            pos = e2 / p.n_w;
-            pr = p.n_t + p.n_h + (e2 - pos * p.n_w);
-        }
-        float sn, cs;
-        sincosf(float(pos) * p.omega[pr], &sn, &cs);
-        tab[e] = make_float2(cs, sn);
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -175,16 +194,18 @@ __global__ void __launch_bounds__(256, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            tma_prefetch_desc(&tm_cc);
-            tma_prefetch_desc(&tm_cr);
-            tma_prefetch_desc(&tm_qn);
-            tma_prefetch_desc(&tm_wuk);
-            tma_prefetch_desc(&tm_wuv);
+            for (int r = 0; r < 2; ++r) {
+                tma_prefetch_desc(&maps.cc[r]);
+                tma_prefetch_desc(&maps.kr[r]);
+            }
+            tma_prefetch_desc(&maps.qn);
+            tma_prefetch_desc(&maps.wuk);
+            tma_prefetch_desc(&maps.wuv);
             mbar_arrive_expect_tx(&bar->q_full, C::QN_BYTES + C::WUK_BYTES);
             for (int c = 0; c < C::QN_CHUNKS; ++c)
-                tma_load_4d(stage(NS - 2) + c * BM * 32, &tm_qn, &bar->q_full, c * 16, h, q0, b);
+                tma_load_4d(stage(NS - 2) + c * BM * 32, &maps.qn, &bar->q_full, c * 16, h, q0, b);
             for (int a = 0; a < C::C_ATOMS; ++a)
-                tma_load_2d(stage(NS - 1) + a * C::WUK_ATOM, &tm_wuk, &bar->q_full, a * 64, h * DN);
+                tma_load_2d(stage(NS - 1) + a * C::WUK_ATOM, &maps.wuk, &bar->q_full, a * 64, h * DN);
             int issued = 0;
             bool qabs_seen = false;
             for (int j = 0; j <= nt; ++j) {
@@ -197,16 +218,16 @@ __global__ void __launch_bounds__(256, 1)
                 }
                 if (!ok) break;
                 if (j < nt) {
-                    int start, valid;
-                    key_tile<BK>(p, j, start, valid);
+                    int run, row, valid;
+                    key_tile<BK>(p, j, run, row, valid);
                     mbar_arrive_expect_tx(&bar->full[s], C::STAGE);
                     for (int a = 0; a < C::C_ATOMS; ++a)
-                        tma_load_3d(stage(s) + a * C::C_ATOM, &tm_cc, &bar->full[s], a * 64, start, b);
-                    tma_load_3d(stage(s) + C::C_ATOMS * C::C_ATOM, &tm_cr, &bar->full[s], DC, start, b);
+                        tma_load_3d(stage(s) + a * C::C_ATOM, &maps.cc[run], &bar->full[s], a * 64, row, b);
+                    tma_load_3d(stage(s) + C::C_ATOMS * C::C_ATOM, &maps.kr[run], &bar->full[s], 0, row, b);
                 } else {
                     mbar_arrive_expect_tx(&bar->full[s], C::WUV_BYTES);
                     for (int a = 0; a < C::C_ATOMS; ++a)
-                        tma_load_2d(stage(s) + a * C::WUV_ATOM, &tm_wuv, &bar->full[s], a * 64, h * DV);
+                        tma_load_2d(stage(s) + a * C::WUV_ATOM, &maps.wuv, &bar->full[s], a * 64, h * DV);
                 }
                 issued = j + 1;
             }
@@ -238,23 +259,21 @@ __global__ void __launch_bounds__(256, 1)
             constexpr uint32_t id_pv = idesc_bf16_f32(128, DC, false, true);
             for (int j = 0; ok && j <= nt; ++j) {
                 if (j < nt) {
-                    // S_j = Q . K_j^T : K = DC latent + DR rope columns, 16 per MMA
+                    // S_j = Q . K_j^T : K = DC latent (bf16) + DR rotated rope (fp16) columns
                     const int s = j % NS;
-                    ok = mbar_wait(&bar->rot[s], (j / NS) & 1, ab, to, 32);
+                    ok = mbar_wait(&bar->full[s], (j / NS) & 1, ab, to, 32);
                     if (ok && j > 0) ok = mbar_wait(&bar->s_free, (j - 1) & 1, ab, to, 33);
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t st = smem_u32(stage(s));
 #pragma unroll
-                    for (int k = 0; k < C::W / 16; ++k) {
-                        if (k < DC / 16)  // latent part: bf16 x bf16
-                            umma_ts(tmem + C::S_COL, tmem + C::Q_COL + k * 8,
-                                    sdesc(st + (k / 4) * C::C_ATOM + (k % 4) * 32, 16, 1024, SW128), id_s, k > 0);
-                        else              // rotated RoPE part: fp16 x fp16
-                            umma_ts(tmem + C::S_COL, tmem + C::Q_COL + k * 8,
-                                    sdesc(st + C::C_ATOMS * C::C_ATOM + (k - DC / 16) * 32, 16, 8 * C::R_ROWB, C::R_SW),
-                                    id_s_rope, 1);
-                    }
+                    for (int k = 0; k < DC / 16; ++k)
+                        umma_ts(tmem + C::S_COL, tmem + C::Q_COL + k * 8,
+                                sdesc(st + (k / 4) * C::C_ATOM + (k % 4) * 32, 16, 1024, SW128), id_s, k > 0);
+#pragma unroll
+                    for (int k = 0; k < DR / 16; ++k)
+                        umma_ts(tmem + C::S_COL, tmem + C::Q_COL + DC / 2 + k * 8,
+                                sdesc(st + C::C_ATOMS * C::C_ATOM + k * 32, 16, 8 * C::R_ROWB, C::R_SW), id_s_rope, 1);
                     umma_commit(&bar->s_full);
                 }
                 if (j > 0) {
@@ -297,48 +316,12 @@ __global__ void __launch_bounds__(256, 1)
                 mbar_wait_drain(&bar->drain, 0, to);
             }
         }
-    } else if (warp < 4) {
-        // ------------------------------------------------------------ RoPE transform
-        const int tid = threadIdx.x - 64;
-        constexpr int CHUNKS = C::R_ROWB / 16;
-        for (int j = 0; j < nt; ++j) {
-            const int s = j % NS;
-            if (!__all_sync(0xffffffffu, mbar_wait(&bar->full[s], (j / NS) & 1, ab, to, 20))) break;
-            int start, valid;
-            key_tile<BK>(p, j, start, valid);
-            uint8_t* kr = stage(s) + C::C_ATOMS * C::C_ATOM;
-            for (int rr = tid; rr < BK; rr += 64) {
-                if (rr < valid) {
-                    const int R = start + rr;
-                    const int slot = R / p.T_f;
-                    const int pp = R - slot * p.T_f;
-                    int t = slot - p.oldest;
-                    if (t < 0) t += p.slots;
-                    const int hh = pp / p.grid_w;
-                    const int ww = pp - hh * p.grid_w;
-                    uint8_t* row = kr + rr * C::R_ROWB;
-                    const int sw = (rr * C::R_ROWB >> 7) & (CHUNKS - 1);
-#pragma unroll
-                    for (int c = 0; c < CHUNKS; ++c) {
-                        uint4* ptr = reinterpret_cast<uint4*>(row + ((c ^ sw) << 4));
-                        uint4 v = *ptr;
-                        v.x = rotate_pair(v.x, rope_cs(tab, p, 4 * c + 0, t, hh, ww));
-                        v.y = rotate_pair(v.y, rope_cs(tab, p, 4 * c + 1, t, hh, ww));
-                        v.z = rotate_pair(v.z, rope_cs(tab, p, 4 * c + 2, t, hh, ww));
-                        v.w = rotate_pair(v.w, rope_cs(tab, p, 4 * c + 3, t, hh, ww));
-                        *ptr = v;
-                    }
-                }
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar->rot[s]);
-        }
     } else {
         // ------------------------------------------------------------ softmax / epilogue
-        const int w4 = warp - 4;
+        // warps 2-5; a warp may only touch TMEM lanes 32 (warp % 4) .. + 31
+        const int w4 = warp & 3;
         const int quad = lane & 3;
-        const uint32_t tl = tmem + (uint32_t(w4 * 32) << 16);  // this warp's TMEM lane quarter
+        const uint32_t tl = tmem + (uint32_t(w4 * 32) << 16);
         const uint32_t tl16 = tl + (16u << 16);
         const float sl = p.scale_log2;
 
@@ -370,10 +353,10 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
                 for (int c = 0; c < DR / 8; ++c) {
                     const uint4 v = __ldg(src + c);
-                    qr[4 * c + 0] = rotate_pair(v.x, rope_cs(tab, p, 4 * c + 0, tq, hq, wq));
-                    qr[4 * c + 1] = rotate_pair(v.y, rope_cs(tab, p, 4 * c + 1, tq, hq, wq));
-                    qr[4 * c + 2] = rotate_pair(v.z, rope_cs(tab, p, 4 * c + 2, tq, hq, wq));
-                    qr[4 * c + 3] = rotate_pair(v.w, rope_cs(tab, p, 4 * c + 3, tq, hq, wq));
+                    qr[4 * c + 0] = rotate_pair(v.x, rope_theta(p, 4 * c + 0, tq, hq, wq));
+                    qr[4 * c + 1] = rotate_pair(v.y, rope_theta(p, 4 * c + 1, tq, hq, wq));
+                    qr[4 * c + 2] = rotate_pair(v.z, rope_theta(p, 4 * c + 2, tq, hq, wq));
+                    qr[4 * c + 3] = rotate_pair(v.w, rope_theta(p, 4 * c + 3, tq, hq, wq));
                 }
             }
             if constexpr (DR == 16) {
@@ -412,9 +395,9 @@ __global__ void __launch_bounds__(256, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar->s_free);
 
-            int start, valid;
-            key_tile<BK>(p, j, start, valid);
-            if (valid < BK) {  // ragged last tile of a segment: mask the missing keys
+            int run, row, valid;
+            key_tile<BK>(p, j, run, row, valid);
+            if (valid < BK) {  // ragged last tile of a run: mask the missing keys
 #pragma unroll
                 for (int c = 0; c < 2; ++c)
 #pragma unroll
@@ -466,7 +449,7 @@ __global__ void __launch_bounds__(256, 1)
                         m_used[k] = mn;
                         l_part[k] *= f[k];
                     }
-#pragma unroll 1
+#pragma unroll
                     for (int half = 0; half < 2; ++half) {
                         const uint32_t base = half ? tl16 : tl;
                         const float fa = f[2 * half], fb = f[2 * half + 1];
@@ -543,7 +526,7 @@ __global__ void __launch_bounds__(256, 1)
             // (nt+1) % NS and (nt+2) % NS (both drained: every PV has completed)
             uint8_t* ol = stage((nt + 1) % NS);
             uint8_t* ol2 = stage((nt + 2) % NS);
-#pragma unroll 1
+#pragma unroll
             for (int half = 0; half < 2; ++half) {
                 const uint32_t base = half ? tl16 : tl;
                 const int r_top = w4 * 32 + half * 16 + (lane >> 2);

@@ -54,7 +54,8 @@ CUtensorMapSwizzle swizzle_of(int bytes) {
 // bf16 tensor map of rank ``rank``: dims/box innermost first, strides in bytes
 // of dims 1..rank-1.
 bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
-              const uint32_t* box, int swizzle_bytes) {
+              const uint32_t* box, int swizzle_bytes,
+              CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t d[5], s[4];
@@ -65,7 +66,7 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, 
         es[i] = 1;
         if (i + 1 < rank) s[i] = strides[i];
     }
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), d, s, bx, es,
+    return fn(m, dtype, rank, const_cast<void*>(base), d, s, bx, es,
               CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_of(swizzle_bytes), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -156,10 +157,27 @@ int run_cache_write(const videomla_dims* d, const void* x, int B, int n_tok, con
 // ----------------------------------------------------------------------------
 // attention
 // ----------------------------------------------------------------------------
+// Valid physical rows of the window: one run, or two when the ring wraps.
+void window_runs(const videomla_window* win, int T_f, int seg_start[2], int seg_len[2]) {
+    seg_start[1] = seg_len[1] = 0;
+    if (win->n_valid == win->slots) {
+        seg_start[0] = 0;
+        seg_len[0] = win->slots * T_f;
+        return;
+    }
+    const int last = win->oldest_slot + win->n_valid;
+    seg_start[0] = win->oldest_slot * T_f;
+    seg_len[0] = (last <= win->slots ? win->n_valid : win->slots - win->oldest_slot) * T_f;
+    if (last > win->slots) {
+        seg_start[1] = 0;
+        seg_len[1] = (last - win->slots) * T_f;
+    }
+}
+
 template <int DC, int DR, int DN, int DV>
 int run_attention(const videomla_dims* d, const void* q_nope, const void* q_rope, const void* W_uk, const void* W_uv,
                   const void* cache, const videomla_window* win, int B, int Nq, void* out, float* lse,
-                  cudaStream_t st) {
+                  void* workspace, cudaStream_t st) {
     using C = vmla::AttnCfg<DC, DR, DN, DV>;
     const int T_f = d->grid_h * d->grid_w;
     const int H = d->n_heads;
@@ -172,35 +190,18 @@ int run_attention(const videomla_dims* d, const void* q_nope, const void* q_rope
     p.grid_w = d->grid_w;
     p.slots = win->slots;
     p.oldest = win->oldest_slot;
-    // valid physical rows of the window: one run, or two when the ring wraps
-    if (win->n_valid == win->slots) {
-        p.seg_start[0] = 0;
-        p.seg_len[0] = rows;
-    } else {
-        const int last = win->oldest_slot + win->n_valid;
-        p.seg_start[0] = win->oldest_slot * T_f;
-        p.seg_len[0] = (last <= win->slots ? win->n_valid : win->slots - win->oldest_slot) * T_f;
-        if (last > win->slots) {
-            p.seg_start[1] = 0;
-            p.seg_len[1] = (last - win->slots) * T_f;
-        }
-    }
+    window_runs(win, T_f, p.seg_start, p.seg_len);
     p.n_kt = (p.seg_len[0] + C::BK - 1) / C::BK + (p.seg_len[1] + C::BK - 1) / C::BK;
     p.q_first = win->n_valid * T_f - Nq;
     p.n_t = d->pairs_t;
     p.n_h = d->pairs_h;
-    p.n_w = d->pairs_w;
-    p.tab_h_off = win->slots * p.n_t;
-    p.tab_w_off = p.tab_h_off + d->grid_h * p.n_h;
-    p.tab_total = p.tab_w_off + d->grid_w * p.n_w;
-    if (p.tab_total > vmla::kAttnTableMax) return VIDEOMLA_EUNSUPPORTED;
     // rope frequencies: an axis owning D_a dims of a full (d_nope + d_rope)-dim
     // head (h, w: floor(n/3) pairs each, t: the rest) uses base^(-2k / D_a)
     {
         const int n_full = (d->d_nope + d->d_rope) / 2;
         const int full_hw = n_full / 3;
         const int full_t = n_full - 2 * full_hw;
-        const int cnt[3] = {p.n_t, p.n_h, p.n_w};
+        const int cnt[3] = {d->pairs_t, d->pairs_h, d->pairs_w};
         const int D[3] = {2 * full_t, 2 * full_hw, 2 * full_hw};
         int pr = 0;
         for (int a = 0; a < 3; ++a)
@@ -213,38 +214,53 @@ int run_attention(const videomla_dims* d, const void* q_nope, const void* q_rope
     p.lse = lse;
     p.timeout_ns = g_timeout_ns.load();
 
-    CUtensorMap tcc, tcr, tqn, tuk, tuv;
-    {
-        const uint64_t dims[3] = {uint64_t(C::W), uint64_t(rows), uint64_t(B)};
-        const uint64_t str[2] = {uint64_t(C::W) * 2, uint64_t(rows) * C::W * 2};
-        const uint32_t box_c[3] = {64, uint32_t(C::BK), 1};
-        const uint32_t box_r[3] = {uint32_t(DR), uint32_t(C::BK), 1};
-        if (!make_map(&tcc, cache, 3, dims, str, box_c, 128)) return VIDEOMLA_ECUDA;
-        if (!make_map(&tcr, cache, 3, dims, str, box_r, DR * 2)) return VIDEOMLA_ECUDA;
+    vmla::AttnMaps maps;
+    const auto* cache_b = static_cast<const __nv_bfloat16*>(cache);
+    const auto* krot = static_cast<const __half*>(workspace);
+    for (int r = 0; r < 2; ++r) {
+        const int run = p.seg_len[r] > 0 ? r : 0;  // an empty second run reuses the first (never read)
+        const uint64_t dc[3] = {uint64_t(C::W), uint64_t(p.seg_len[run]), uint64_t(B)};
+        const uint64_t sc[2] = {uint64_t(C::W) * 2, uint64_t(rows) * C::W * 2};
+        const uint32_t bc[3] = {64, uint32_t(C::BK), 1};
+        if (!make_map(&maps.cc[r], cache_b + size_t(p.seg_start[run]) * C::W, 3, dc, sc, bc, 128))
+            return VIDEOMLA_ECUDA;
+        const uint64_t dr[3] = {uint64_t(DR), uint64_t(p.seg_len[run]), uint64_t(B)};
+        const uint64_t sr[2] = {uint64_t(DR) * 2, uint64_t(rows) * DR * 2};
+        const uint32_t br[3] = {uint32_t(DR), uint32_t(C::BK), 1};
+        if (!make_map(&maps.kr[r], krot + size_t(p.seg_start[run]) * DR, 3, dr, sr, br, DR * 2,
+                      CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+            return VIDEOMLA_ECUDA;
     }
     {
         const uint64_t dims[4] = {uint64_t(DN), uint64_t(H), uint64_t(Nq), uint64_t(B)};
         const uint64_t str[3] = {uint64_t(DN) * 2, uint64_t(H) * DN * 2, uint64_t(Nq) * H * DN * 2};
         const uint32_t box[4] = {16, 1, uint32_t(C::BM), 1};
-        if (!make_map(&tqn, q_nope, 4, dims, str, box, 32)) return VIDEOMLA_ECUDA;
+        if (!make_map(&maps.qn, q_nope, 4, dims, str, box, 32)) return VIDEOMLA_ECUDA;
     }
     {
         const uint64_t dims[2] = {uint64_t(DC), uint64_t(H) * DN};
         const uint64_t str[1] = {uint64_t(DC) * 2};
         const uint32_t box[2] = {64, uint32_t(DN)};
-        if (!make_map(&tuk, W_uk, 2, dims, str, box, 128)) return VIDEOMLA_ECUDA;
+        if (!make_map(&maps.wuk, W_uk, 2, dims, str, box, 128)) return VIDEOMLA_ECUDA;
     }
     {
         const uint64_t dims[2] = {uint64_t(DC), uint64_t(H) * DV};
         const uint64_t str[1] = {uint64_t(DC) * 2};
         const uint32_t box[2] = {64, uint32_t(DV)};
-        if (!make_map(&tuv, W_uv, 2, dims, str, box, 128)) return VIDEOMLA_ECUDA;
+        if (!make_map(&maps.wuv, W_uv, 2, dims, str, box, 128)) return VIDEOMLA_ECUDA;
     }
+    // 1) form the window: rotated rope keys into the workspace
+    {
+        const long long work = (long long)B * (p.seg_len[0] + p.seg_len[1]) * (DR / 8);
+        const int blocks = int((work + 255) / 256);
+        vmla::rope_window_kernel<DC, DR><<<blocks, 256, 0, st>>>(cache_b, static_cast<__half*>(workspace), p, B);
+    }
+    // 2) latent attention
     auto kern = vmla::attention_kernel<C>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
         return VIDEOMLA_ECUDA;
     dim3 grid((Nq + C::BM - 1) / C::BM, H, B);
-    kern<<<grid, C::THREADS, C::SMEM, st>>>(tcc, tcr, tqn, tuk, tuv, p);
+    kern<<<grid, C::THREADS, C::SMEM, st>>>(maps, p);
     return launch_status(kern, C::SMEM);
 }
 
@@ -280,10 +296,17 @@ int videomla_cache_write(const videomla_dims* dims, const void* x, int batch, in
     return VIDEOMLA_EUNSUPPORTED;
 }
 
+size_t videomla_attention_workspace_size(const videomla_dims* dims, const videomla_window* window, int batch) {
+    if (!dims || !window || batch <= 0 || window->slots <= 0 || dims->grid_h <= 0 || dims->grid_w <= 0 ||
+        dims->d_rope <= 0)
+        return 0;
+    return size_t(batch) * window->slots * size_t(dims->grid_h) * dims->grid_w * dims->d_rope * 2;
+}
+
 int videomla_attention(const videomla_dims* dims, const void* q_nope, const void* q_rope, const void* W_uk,
                        const void* W_uv, const void* cache, const videomla_window* window, int batch, int n_query,
-                       void* out, float* lse, void* stream) {
-    if (!basic_dims_ok(dims) || !q_nope || !q_rope || !W_uk || !W_uv || !cache || !window || !out)
+                       void* out, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+    if (!basic_dims_ok(dims) || !q_nope || !q_rope || !W_uk || !W_uv || !cache || !window || !out || !workspace)
         return VIDEOMLA_EINVAL;
     const videomla_window w = *window;
     if (w.slots <= 0 || w.oldest_slot < 0 || w.oldest_slot >= w.slots || w.n_valid < 1 || w.n_valid > w.slots)
@@ -291,15 +314,17 @@ int videomla_attention(const videomla_dims* dims, const void* q_nope, const void
     const long long T_f = (long long)dims->grid_h * dims->grid_w;
     if (batch <= 0 || batch > 65535 || n_query <= 0 || n_query > w.n_valid * T_f) return VIDEOMLA_EINVAL;
     if ((long long)w.slots * T_f > (1ll << 30) || dims->n_heads > 65535) return VIDEOMLA_EINVAL;
+    if (workspace_bytes < videomla_attention_workspace_size(dims, window, batch)) return VIDEOMLA_EINVAL;
     if (!aligned16(q_nope) || !aligned16(q_rope) || !aligned16(W_uk) || !aligned16(W_uv) || !aligned16(cache) ||
-        !aligned16(out) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+        !aligned16(out) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(lse) & 3u))
         return VIDEOMLA_EINVAL;
     if (int rc = check_device()) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int dc = dims->d_c, dr = dims->d_rope, dn = dims->d_nope, dv = dims->d_v;
 #define VMLA_AT(DC_, DR_, DN_, DV_)                        \
     if (dc == DC_ && dr == DR_ && dn == DN_ && dv == DV_) \
-        return run_attention<DC_, DR_, DN_, DV_>(dims, q_nope, q_rope, W_uk, W_uv, cache, &w, batch, n_query, out, lse, st);
+        return run_attention<DC_, DR_, DN_, DV_>(dims, q_nope, q_rope, W_uk, W_uv, cache, &w, batch, n_query, out, lse, \
+                                                 workspace, st);
     VMLA_AT(192, 32, 96, 128)
     VMLA_AT(192, 16, 112, 128)
     VMLA_AT(192, 64, 64, 128)

@@ -27,6 +27,7 @@ CACHE_RAW_LATENT = 1
 EXPORTED = (
     "videomla_cache_write",
     "videomla_attention",
+    "videomla_attention_workspace_size",
     "videomla_strerror",
     "videomla_device_status",
     "videomla_set_wait_timeout_ns",
@@ -68,8 +69,10 @@ def load_library() -> ctypes.CDLL:
         lib.videomla_cache_write.argtypes = [ctypes.POINTER(CDims), vp, ci, ci, vp, vp, vp, vp, ci, ci, cu, vp]
         lib.videomla_cache_write.restype = ci
         lib.videomla_attention.argtypes = [ctypes.POINTER(CDims), vp, vp, vp, vp, vp, ctypes.POINTER(CWindow),
-                                           ci, ci, vp, vp, vp]
+                                           ci, ci, vp, vp, vp, ctypes.c_size_t, vp]
         lib.videomla_attention.restype = ci
+        lib.videomla_attention_workspace_size.argtypes = [ctypes.POINTER(CDims), ctypes.POINTER(CWindow), ci]
+        lib.videomla_attention_workspace_size.restype = ctypes.c_size_t
         lib.videomla_strerror.argtypes = [ci]
         lib.videomla_strerror.restype = ctypes.c_char_p
         lib.videomla_device_status.argtypes = [ci]
@@ -143,12 +146,22 @@ def cache_write(x: torch.Tensor, W_dkv: torch.Tensor, W_kr: torch.Tensor, gamma:
     return cache
 
 
+def workspace_size(dims: Dims, slots: int, oldest: int, n_valid: int, batch: int) -> int:
+    """Bytes of the attention workspace (the window's rotated RoPE keys)."""
+    cd, win = c_dims(dims), CWindow(slots, oldest, n_valid)
+    return int(load_library().videomla_attention_workspace_size(ctypes.byref(cd), ctypes.byref(win), batch))
+
+
 def attention(q_nope: torch.Tensor, q_rope: torch.Tensor, W_uk: torch.Tensor, W_uv: torch.Tensor,
               cache: torch.Tensor, dims: Dims, slots: int, oldest: int, n_valid: int,
               out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-              want_lse: bool = False, stream=None):
+              want_lse: bool = False, workspace: Optional[torch.Tensor] = None, stream=None):
     """Latent attention of the queries over the window; returns ``out``
-    [B, Nq, H, d_v] (and ``lse`` [B, Nq, H] if requested or given)."""
+    [B, Nq, H, d_v] (and ``lse`` [B, Nq, H] if requested or given).
+
+    ``workspace`` is a device byte buffer of at least ``workspace_size(...)``
+    bytes; if omitted, one is taken from torch's stream-ordered caching
+    allocator for this call."""
     lib = load_library()
     B, Nq, H = q_nope.shape[0], q_nope.shape[1], dims.n_heads
     dev = q_nope.device
@@ -166,8 +179,14 @@ def attention(q_nope: torch.Tensor, q_rope: torch.Tensor, W_uk: torch.Tensor, W_
         _check(lse, "lse", torch.float32, (B, Nq, H), dev)
     cd = c_dims(dims)
     win = CWindow(slots, oldest, n_valid)
+    need = int(lib.videomla_attention_workspace_size(ctypes.byref(cd), ctypes.byref(win), B))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    elif workspace.device != dev or workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace must be a {need}-byte buffer on {dev}")
     rc = lib.videomla_attention(ctypes.byref(cd), _ptr(q_nope), _ptr(q_rope), _ptr(W_uk), _ptr(W_uv),
-                                _ptr(cache), ctypes.byref(win), B, Nq, _ptr(out), _ptr(lse), _stream(stream))
+                                _ptr(cache), ctypes.byref(win), B, Nq, _ptr(out), _ptr(lse), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(stream))
     if rc != OK:
         raise VideoMLAError(rc, "videomla_attention")
     return (out, lse) if lse is not None else out

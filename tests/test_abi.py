@@ -83,7 +83,9 @@ def test_attention_rejects_bad_arguments(lib):
     d = _dims()
     f = lib.videomla_attention
     win = V.CWindow(21, 0, 21)
-    ok_args = [ctypes.byref(d), P, P, P, P, P, ctypes.byref(win), 1, 4680, P, None, None]
+    ws = lib.videomla_attention_workspace_size(ctypes.byref(d), ctypes.byref(win), 1)
+    assert ws == 21 * 1560 * 32 * 2
+    ok_args = [ctypes.byref(d), P, P, P, P, P, ctypes.byref(win), 1, 4680, P, None, P, ws, None]
     def call(**over):
         a = list(ok_args)
         for i, v in over.items():
@@ -98,6 +100,9 @@ def test_attention_rejects_bad_arguments(lib):
     assert call(a8=21 * 1560 + 1) == V.EINVAL             # more queries than window tokens
     assert call(a8=0) == V.EINVAL
     assert call(a10=ctypes.c_void_p(0x10002)) == V.EINVAL  # misaligned lse
+    assert call(a11=None) == V.EINVAL                     # no workspace
+    assert call(a12=ws - 1) == V.EINVAL                   # workspace too small
+    assert call(a11=ctypes.c_void_p(0x10008)) == V.EINVAL  # misaligned workspace
 
 
 def test_valid_call_without_device_reports_no_device(lib):
@@ -106,7 +111,8 @@ def test_valid_call_without_device_reports_no_device(lib):
         pytest.skip("a device is present")
     d = _dims()
     win = V.CWindow(21, 0, 21)
-    rc = lib.videomla_attention(ctypes.byref(d), P, P, P, P, P, ctypes.byref(win), 1, 4680, P, None, None)
+    rc = lib.videomla_attention(ctypes.byref(d), P, P, P, P, P, ctypes.byref(win), 1, 4680, P, None, P,
+                                1 << 30, None)
     assert rc == V.ENODEVICE
     rc = lib.videomla_cache_write(ctypes.byref(d), P, 1, 4680, P, P, None, P, 21, 18, 0, None)
     assert rc == V.ENODEVICE
@@ -120,7 +126,7 @@ def test_unsupported_geometry_is_reported(lib):
     win = V.CWindow(21, 0, 21)
     P2 = ctypes.c_void_p(0x10000)
     assert lib.videomla_attention(ctypes.byref(d), P2, P2, P2, P2, P2, ctypes.byref(win), 1, 16, P2, None,
-                                  None) == V.EUNSUPPORTED
+                                  P2, 1 << 30, None) == V.EUNSUPPORTED
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
