@@ -145,6 +145,42 @@ int videomla_attention(const videomla_dims* dims, const void* q_nope, const void
                        void* out, float* lse, void* workspace, size_t workspace_bytes,
                        void* stream);
 
+/*
+ * Bytes of the library's built-in scratch array used by
+ * videomla_attention_static_workspace (16 MiB per device that loads the library).
+ */
+#define VIDEOMLA_STATIC_WORKSPACE_BYTES (16u << 20)
+
+/*
+ * videomla_attention_static_workspace -- videomla_attention without a caller
+ * workspace.  (No counterpart in the paper: this is an integration aid.)
+ *
+ * For callers that cannot allocate device memory themselves -- for example a
+ * host framework whose memory is owned by a pool or arena it does not expose,
+ * code running where cudaMalloc is not allowed or would break a capture, or a
+ * plug-in that may only use the buffers it is handed.  The window's rotated
+ * RoPE keys go to a fixed scratch array compiled into the library
+ * (VIDEOMLA_STATIC_WORKSPACE_BYTES per device, held from library load until
+ * process exit).  The function itself allocates nothing and frees nothing.
+ *
+ * Arguments, results and arithmetic are those of videomla_attention.
+ * - Sizes: if videomla_attention_workspace_size(dims, window, batch) exceeds
+ *   VIDEOMLA_STATIC_WORKSPACE_BYTES the call returns VIDEOMLA_EINVAL and
+ *   launches nothing.
+ * - Set-up: the first call on each device looks up the device address of the
+ *   scratch array with that device current (cudaGetSymbolAddress), which may
+ *   load the library's kernels; make that first call before any stream capture.
+ * - Sharing: every call on a device uses the same scratch array and leaves the
+ *   last call's contents in it.  Nothing in it needs to start at zero (each call
+ *   rewrites every row it reads).  Calls whose kernels can overlap on the GPU
+ *   (different streams without ordering between them) race on the array; issue
+ *   them on one stream or order them.
+ */
+int videomla_attention_static_workspace(const videomla_dims* dims, const void* q_nope, const void* q_rope,
+                                        const void* W_uk, const void* W_uv, const void* cache,
+                                        const videomla_window* window, int batch, int n_query,
+                                        void* out, float* lse, void* stream);
+
 /* Name of an error code (static string, never NULL). */
 const char* videomla_strerror(int code);
 

@@ -332,6 +332,51 @@ int videomla_attention(const videomla_dims* dims, const void* q_nope, const void
     return VIDEOMLA_EUNSUPPORTED;
 }
 
+}  // extern "C"
+
+// ----------------------------------------------------------------------------
+// videomla_attention_static_workspace: the attention workspace lives in this
+// fixed device array instead of caller memory.  In host code the name below is
+// only a host-side stand-in; its device address comes from cudaGetSymbolAddress.
+// ----------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_static_workspace[VIDEOMLA_STATIC_WORKSPACE_BYTES];
+
+namespace {
+
+// Device address of g_static_workspace on the current device, looked up once
+// per device with that device current.  nullptr if the lookup fails.
+void* static_workspace_address() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    static std::mutex mu;
+    static void* addr[64] = {};
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess) return nullptr;
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+int videomla_attention_static_workspace(const videomla_dims* dims, const void* q_nope, const void* q_rope,
+                                        const void* W_uk, const void* W_uv, const void* cache,
+                                        const videomla_window* window, int batch, int n_query, void* out, float* lse,
+                                        void* stream) {
+    if (!dims || !window || batch <= 0) return VIDEOMLA_EINVAL;
+    const size_t need = videomla_attention_workspace_size(dims, window, batch);
+    if (need == 0 || need > VIDEOMLA_STATIC_WORKSPACE_BYTES) return VIDEOMLA_EINVAL;
+    if (int rc = check_device()) return rc;
+    void* ws = static_workspace_address();
+    if (ws == nullptr) return VIDEOMLA_ECUDA;
+    return videomla_attention(dims, q_nope, q_rope, W_uk, W_uv, cache, window, batch, n_query, out, lse, ws,
+                              VIDEOMLA_STATIC_WORKSPACE_BYTES, stream);
+}
+
 const char* videomla_strerror(int code) {
     switch (code) {
         case VIDEOMLA_OK: return "ok";

@@ -28,6 +28,7 @@ EXPORTED = (
     "videomla_cache_write",
     "videomla_attention",
     "videomla_attention_workspace_size",
+    "videomla_attention_static_workspace",
     "videomla_strerror",
     "videomla_device_status",
     "videomla_set_wait_timeout_ns",
