@@ -84,11 +84,10 @@ def ncu_traffic(kernel: str):
         e = t.get(kernel)
         if not e:
             return None
-        from mla_latent_kv_write_b200 import build as vb
         import hashlib
         h = hashlib.sha256()
-        for s in vb.SOURCES:
-            with open(s, "rb") as fh:
+        for s in e["sources"]:
+            with open(os.path.join(ROOT, s), "rb") as fh:
                 h.update(fh.read())
         if e.get("sources_sha256") != h.hexdigest():
             return None
