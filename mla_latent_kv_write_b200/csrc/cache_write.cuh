@@ -4,12 +4,22 @@
 // the latent part (App. D.2), bf16 rows written into the FIFO frame ring
 // (App. D.4).  k^R is stored unrotated and unnormalised.
 //
-// One CTA per (128-token tile, batch element); 192 threads:
+// One thread-block cluster of ``ksplit`` CTAs (1 to 4) per 128-token tile;
+// CTA r of the cluster accumulates the K range [r, r+1) * d_model / ksplit.
+// 192 threads per CTA:
 //   warp 0     TMA producer (x tile 128 x 64 and W tile N x 64 per stage)
 //   warp 1     tcgen05.mma issuer (M = 128, N = d_c + d_rope, K = 16 steps)
 //              and tensor-memory owner
-//   warps 2-5  epilogue: one TMEM lane (token) per thread, RMSNorm in fp32,
-//              bf16 RNE, 16-byte stores into the ring rows
+//   warps 2-5  epilogue.  After a cluster barrier (every CTA's MMAs are done,
+//              so every CTA's pipeline stages are free) each thread copies one
+//              TMEM lane (token row) of its fp32 partial into local shared
+//              memory; one thread then ships each peer the contiguous block of
+//              the rows that peer owns (rows [128 r / ksplit, 128 (r+1) / ksplit)
+//              belong to rank r) with one bulk shared-to-shared copy completing
+//              on the peer's mbarrier.  Each owner sums the ksplit partials of its
+//              rows, one warp per row (lane l holds columns 8l .. 8l+7), reduces
+//              the row's sum of squares with warp shuffles, applies RMSNorm and
+//              writes the row as 16-byte bf16 stores.
 #pragma once
 
 #include "ptx.cuh"
@@ -19,6 +29,7 @@ namespace vmla {
 struct CacheWriteParams {
     int n_tok;            // tokens per batch element in this call
     int d_model;
+    int ksplit;           // CTAs per cluster along K (1 to 4)
     int T_f;              // tokens per latent frame
     int slots;            // ring capacity in frames
     int first_slot;       // slot of frame 0 of the chunk
@@ -32,7 +43,7 @@ struct CacheWriteParams {
 template <int DC, int DR>
 struct CacheWriteCfg {
     static constexpr int N = DC + DR;                 // cached scalars per token
-    static constexpr int BM = 128;                    // tokens per CTA
+    static constexpr int BM = 128;                    // tokens per tile
     static constexpr int BKK = 64;                    // K elements per stage (one 128-B swizzle row)
     static constexpr int N_MMA = N <= 256 ? 1 : 2;    // MMA column chunks
     static constexpr int N_CHUNK = N / N_MMA;
@@ -42,11 +53,23 @@ struct CacheWriteCfg {
     static constexpr int STAGE = X_BYTES + W_BYTES;
     static constexpr int WBOX = DC <= 192 ? DC : 192; // rows per W_dkv TMA box
     static constexpr int TMEM_COLS = N <= 256 ? 256 : 512;
-    static constexpr int SMEM = NS * STAGE + 1024 + 256;
+    static constexpr int RED_STRIDE = N + 4;          // fp32 words per partial row (bank-conflict pad)
+    static constexpr int PART_BYTES = BM * RED_STRIDE * 4;               // this CTA's fp32 partial
+    static constexpr int SMEM_LIMIT = 232448;                            // opt-in shared memory per CTA
+    // rows received from the peers for a K split ks: (ks - 1) * ceil(128 / ks)
+    static constexpr int recv_rows(int ks) { return (ks - 1) * ((BM + ks - 1) / ks); }
+    static constexpr bool fits(int ks) {
+        return PART_BYTES + recv_rows(ks) * RED_STRIDE * 4 + 1024 + 256 <= SMEM_LIMIT;
+    }
+    static constexpr int KS_MAX = N > 256 ? 1 : fits(4) ? 4 : fits(3) ? 3 : fits(2) ? 2 : 1;  // cluster size
+    static constexpr int RED_BYTES = PART_BYTES + recv_rows(KS_MAX) * RED_STRIDE * 4;
+    static constexpr int BUF = NS * STAGE > RED_BYTES ? NS * STAGE : RED_BYTES;
+    static constexpr int SMEM = BUF + 1024 + 256;
+    static_assert(SMEM <= SMEM_LIMIT, "shared memory");
     static constexpr int THREADS = 192;
     static_assert(N % 16 == 0 && N_CHUNK % 16 == 0 && N_CHUNK <= 256, "MMA N");
     static_assert(DC % 32 == 0 && DR % 16 == 0 && DC % WBOX == 0, "widths");
-    static_assert((N * 2) % 16 == 0, "cache row must be 16-byte aligned");
+    static_assert(N % 8 == 0 && N / 8 <= 64 && DC % 8 == 0, "a warp covers a row in 8-column groups");
 };
 
 template <int DC, int DR>
@@ -54,18 +77,25 @@ __global__ void __launch_bounds__(192, 1)
     cache_write_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_wdkv,
                        const __grid_constant__ CUtensorMap tm_wkr, const CacheWriteParams p) {
     using C = CacheWriteCfg<DC, DR>;
+    constexpr int N = C::N;
+    constexpr int GROUPS = N / 8;              // 8-column groups of a row
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::NS * C::STAGE);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BUF);
     uint64_t* empty = full + C::NS;
     uint64_t* done = empty + C::NS;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    uint64_t* recv = done + 1;  // partials of the peers for the rows this CTA owns
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recv + 1);
     AbortState* ab = reinterpret_cast<AbortState*>(tmem_slot + 1);
+    float* part = reinterpret_cast<float*>(smem);  // fp32 partial [BM][RED_STRIDE], reuses the stages
+    float* rbuf = reinterpret_cast<float*>(smem + C::PART_BYTES);  // [ks-1][rows_max][RED_STRIDE]
 
     const int warp = warp_id(), lane = lane_id();
     const int row0 = blockIdx.x * C::BM;
-    const int b = blockIdx.y;
-    const int k_chunks = p.d_model / C::BKK;
+    const int b = blockIdx.z;
+    const uint32_t rank = cluster_ctarank();
+    const int k_chunks = p.d_model / C::BKK / p.ksplit;
+    const int kc0 = int(rank) * k_chunks;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::NS; ++s) {
@@ -73,7 +103,12 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(&empty[s], 1);
         }
         mbar_init(done, 1);
+        mbar_init(recv, 1);
         ab->flag = 0;
+        if (p.ksplit > 1) {  // bytes the peers will send for this CTA's rows
+            const int rows_mine = (C::BM * (int(rank) + 1)) / p.ksplit - (C::BM * int(rank)) / p.ksplit;
+            mbar_arrive_expect_tx(recv, uint32_t((p.ksplit - 1) * rows_mine * C::RED_STRIDE * 4));
+        }
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -97,11 +132,11 @@ __global__ void __launch_bounds__(192, 1)
             for (int kc = 0; kc < k_chunks; ++kc) {
                 const int s = kc % C::NS;
                 if (kc >= C::NS && !mbar_wait(&empty[s], ((kc / C::NS) - 1) & 1, ab, p.timeout_ns, 1)) break;
+                const int kx = (kc0 + kc) * C::BKK;
                 mbar_arrive_expect_tx(&full[s], C::STAGE);
-                tma_load_3d(stage_x(s), &tm_x, &full[s], kc * C::BKK, row0, b);
-                for (int r = 0; r < DC; r += C::WBOX)
-                    tma_load_2d(stage_w(s) + r * 128, &tm_wdkv, &full[s], kc * C::BKK, r);
-                tma_load_2d(stage_w(s) + DC * 128, &tm_wkr, &full[s], kc * C::BKK, 0);
+                tma_load_3d(stage_x(s), &tm_x, &full[s], kx, row0, b);
+                for (int r = 0; r < DC; r += C::WBOX) tma_load_2d(stage_w(s) + r * 128, &tm_wdkv, &full[s], kx, r);
+                tma_load_2d(stage_w(s) + DC * 128, &tm_wkr, &full[s], kx, 0);
                 issued = kc + 1;
             }
             if (ab->flag) {  // let the copies still in flight land before the CTA exits
@@ -135,66 +170,139 @@ __global__ void __launch_bounds__(192, 1)
             umma_commit(done);
             if (!ok) mbar_wait_drain(done, 0, p.timeout_ns);  // no MMA may be in flight at teardown
         }
-    } else {
-        // epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31
-        const int quarter = warp & 3;
-        const int r = quarter * 32 + lane;
-        const int token = row0 + r;
-        const bool valid = token < p.n_tok;
-        const uint32_t trow = tmem + (uint32_t(quarter * 32) << 16);
-        const bool go = __all_sync(0xffffffffu, mbar_wait(done, 0, ab, p.timeout_ns, 3) && !ab->flag);
+    }
+
+    // epilogue warps: the MMAs of this CTA are complete before the cluster barrier
+    const int quarter = warp & 3;
+    const uint32_t trow = tmem + (uint32_t(quarter * 32) << 16);
+    bool go = true;
+    if (warp >= 2) go = __all_sync(0xffffffffu, mbar_wait(done, 0, ab, p.timeout_ns, 3) && !ab->flag);
+
+    // every thread of every CTA of the cluster takes this barrier: after it every
+    // CTA's pipeline stages are free to receive partials
+    tc_fence_before();
+    cluster_sync();
+
+    // abort flags of the peers (no peer can finish before it has received our rows)
+    bool any_abort = false;
+    for (int k = 0; k < p.ksplit; ++k)
+        any_abort |= ld_dsmem_s32(mapa_shared(smem_u32(const_cast<int*>(&ab->flag)), uint32_t(k))) != 0;
+
+    const int rows_max = (C::BM + p.ksplit - 1) / p.ksplit;
+    if (warp >= 2) {
+        // (a) TMEM lane (token row) r -> part[r][0 .. N), 128 columns per wait
         if (go) {
             tc_fence_after();
-            __nv_bfloat16* dst = nullptr;
-            if (valid) {
-                const int frame = token / p.T_f;
-                const int slot = (p.first_slot + frame) % p.slots;
-                const long long row = (long long)b * p.slots * p.T_f + (long long)slot * p.T_f + (token - frame * p.T_f);
-                dst = p.cache + row * C::N;
-            }
-            float rstd = 1.0f;
-            uint32_t v[32];
-            if (p.normalize) {
-                float ss = 0.f;
+            const int r = quarter * 32 + lane;
+            float* dst = part + r * C::RED_STRIDE;
 #pragma unroll 1
-                for (int c = 0; c < DC; c += 32) {
-                    tmem_ld_32x32b_x32(trow + c, v);
-                    tmem_wait_ld();
+            for (int c0 = 0; c0 < N; c0 += 128) {
+                uint32_t v[4][32];
+                const int nc = N - c0 < 128 ? N - c0 : 128;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float f = __uint_as_float(v[i]);
-                        ss = fmaf(f, f, ss);
-                    }
-                }
-                rstd = rsqrtf(ss * (1.0f / DC) + p.eps);
-            }
-#pragma unroll 1
-            for (int c = 0; c < C::N; c += 32) {
-                const int ncol = (C::N - c) < 32 ? 16 : 32;  // DR may leave a 16-column tail
-                if (ncol == 32) {
-                    tmem_ld_32x32b_x32(trow + c, v);
-                } else {
-                    uint32_t (&v16)[16] = *reinterpret_cast<uint32_t (*)[16]>(v);
-                    tmem_ld_32x32b_x16(trow + c, v16);
+                for (int q = 0; q < 4; ++q) {
+                    if (32 * q + 32 <= nc) tmem_ld_32x32b_x32(trow + c0 + 32 * q, v[q]);
+                    else if (32 * q + 16 <= nc) tmem_ld_32x32b_x16(trow + c0 + 32 * q, *reinterpret_cast<uint32_t (*)[16]>(v[q]));
                 }
                 tmem_wait_ld();
-                uint32_t packed[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    float a = __uint_as_float(v[2 * i]), bb = __uint_as_float(v[2 * i + 1]);
-                    const int col = c + 2 * i;
-                    if (col < DC && p.normalize) {
-                        const float g0 = p.gamma ? __ldg(p.gamma + col) : 1.f;
-                        const float g1 = p.gamma ? __ldg(p.gamma + col + 1) : 1.f;
-                        a = a * rstd * g0;
-                        bb = bb * rstd * g1;
-                    }
-                    packed[i] = pack_bf16(a, bb);
+                for (int q = 0; q < 4; ++q)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        if (32 * q + 4 * e + 4 <= nc)
+                            *reinterpret_cast<float4*>(dst + c0 + 32 * q + 4 * e) =
+                                make_float4(__uint_as_float(v[q][4 * e]), __uint_as_float(v[q][4 * e + 1]),
+                                            __uint_as_float(v[q][4 * e + 2]), __uint_as_float(v[q][4 * e + 3]));
+            }
+        }
+        fence_proxy_async_smem();  // the bulk copies read part through the async proxy
+        named_barrier_sync(1, 128);
+        // (b) ship each peer the contiguous block of its rows: one bulk copy per peer
+        if (warp == 2 && lane == 0 && p.ksplit > 1) {
+            for (int k = 0; k < p.ksplit; ++k) {
+                if (k == int(rank)) continue;
+                const int lo = (C::BM * k) / p.ksplit, hi = (C::BM * (k + 1)) / p.ksplit;
+                const int slot = int(rank) < k ? int(rank) : int(rank) - 1;
+                const uint32_t dst = mapa_shared(smem_u32(rbuf + slot * rows_max * C::RED_STRIDE), uint32_t(k));
+                bulk_copy_to_peer(dst, smem_u32(part + lo * C::RED_STRIDE), uint32_t((hi - lo) * C::RED_STRIDE * 4),
+                                  mapa_shared(smem_u32(recv), uint32_t(k)));
+            }
+            bulk_commit();
+        }
+        // our outgoing copies must have read ``part`` before this CTA exits
+        if (warp == 2 && lane == 0 && p.ksplit > 1) bulk_wait_read();
+    }
+
+    // (c) all 192 threads: sum the ksplit partials of this CTA's rows, RMSNorm,
+    // bf16 rows.  Four threads per row (a quad of lanes); thread q of the quad
+    // holds the 8-column groups q, q + 4, ... so that each step of the quad
+    // covers 128 contiguous bytes.  The row's sum of squares is reduced over the
+    // quad with warp shuffles.
+    const bool got = p.ksplit == 1 || __all_sync(0xffffffffu, mbar_wait(recv, 0, ab, p.timeout_ns, 4));
+    const int r_lo = (C::BM * int(rank)) / p.ksplit, r_hi = (C::BM * (int(rank) + 1)) / p.ksplit;
+    const int q = threadIdx.x & 3;
+    constexpr int GPT = (GROUPS + 3) / 4;  // groups per thread
+    float g[GPT][8];
+#pragma unroll
+    for (int i = 0; i < GPT; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int col = 8 * (q + 4 * i) + e;
+            g[i][e] = (p.gamma != nullptr && col < DC) ? __ldg(p.gamma + col) : 1.0f;
+        }
+    const bool store = got && !any_abort && !ab->flag;
+    for (int r0 = r_lo; r0 < r_hi; r0 += C::THREADS / 4) {  // warp-uniform trip count
+        const int r = r0 + int(threadIdx.x >> 2);
+        const int token = row0 + r;
+        const bool live = store && r < r_hi && token < p.n_tok;
+        float a[GPT][8];
+#pragma unroll
+        for (int i = 0; i < GPT; ++i) {
+            const int grp = q + 4 * i;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) a[i][e] = 0.f;
+            if (live && grp < GROUPS) {
+                const float* src = part + r * C::RED_STRIDE + 8 * grp;
+                float4 u = *reinterpret_cast<const float4*>(src), w = *reinterpret_cast<const float4*>(src + 4);
+                a[i][0] = u.x; a[i][1] = u.y; a[i][2] = u.z; a[i][3] = u.w;
+                a[i][4] = w.x; a[i][5] = w.y; a[i][6] = w.z; a[i][7] = w.w;
+                for (int sl = 0; sl + 1 < p.ksplit; ++sl) {
+                    const float* sk = rbuf + (sl * rows_max + (r - r_lo)) * C::RED_STRIDE + 8 * grp;
+                    u = *reinterpret_cast<const float4*>(sk);
+                    w = *reinterpret_cast<const float4*>(sk + 4);
+                    a[i][0] += u.x; a[i][1] += u.y; a[i][2] += u.z; a[i][3] += u.w;
+                    a[i][4] += w.x; a[i][5] += w.y; a[i][6] += w.z; a[i][7] += w.w;
                 }
-                if (valid) {
-                    uint4* d4 = reinterpret_cast<uint4*>(dst + c);
-                    for (int q = 0; q < ncol / 8; ++q)
-                        d4[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+            }
+        }
+        float scale = 1.0f;
+        if (p.normalize) {
+            float ss = 0.f;
+#pragma unroll
+            for (int i = 0; i < GPT; ++i)
+                if (q + 4 * i < DC / 8) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) ss = fmaf(a[i][e], a[i][e], ss);
+                }
+            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+            ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+            scale = rsqrtf(ss * (1.0f / DC) + p.eps);
+        }
+        if (live) {
+            const int frame = token / p.T_f;
+            const int slot = (p.first_slot + frame) % p.slots;
+            const long long row = (long long)b * p.slots * p.T_f + (long long)slot * p.T_f + (token - frame * p.T_f);
+            uint4* out = reinterpret_cast<uint4*>(p.cache + row * N);
+#pragma unroll
+            for (int i = 0; i < GPT; ++i) {
+                const int grp = q + 4 * i;
+                if (grp < GROUPS) {
+                    const bool norm = p.normalize && grp < DC / 8;
+                    float o[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) o[e] = norm ? a[i][e] * scale * g[i][e] : a[i][e];
+                    out[grp] = make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]),
+                                          pack_bf16(o[6], o[7]));
                 }
             }
         }

@@ -111,6 +111,54 @@ bool basic_dims_ok(const videomla_dims* d) {
 // ----------------------------------------------------------------------------
 // cache_write
 // ----------------------------------------------------------------------------
+// K split of the cache write: CTAs per cluster (1-4) dividing the K chunks.
+// Clusters are placed inside one GPC, so the number that fit at once
+// (cudaOccupancyMaxActiveClusters) decides the waves; pick the split with the
+// least work per SM = waves * chunks / ksplit (cached per device and shape).
+template <class K>
+int pick_ksplit(K kern, int threads, int smem, int chunks, int clusters, int max_split) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static std::mutex mu;
+    static int cache[64][5] = {};  // max active clusters per (device, ksplit)
+    int best = 1;
+    long long best_cost = -1;
+    for (int k = max_split; k >= 1; --k) {
+        if (chunks % k != 0) continue;
+        int active = 0;
+        {
+            std::lock_guard<std::mutex> lock(mu);
+            if (dev >= 0 && dev < 64 && cache[dev][k] > 0) active = cache[dev][k];
+        }
+        if (active == 0) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(clusters, k, 1);
+            cfg.blockDim = dim3(threads);
+            cfg.dynamicSmemBytes = smem;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 1;
+            attr[0].val.clusterDim.y = k;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) != cudaSuccess || active <= 0) {
+                cudaGetLastError();
+                continue;
+            }
+            std::lock_guard<std::mutex> lock(mu);
+            if (dev >= 0 && dev < 64) cache[dev][k] = active;
+        }
+        const long long waves = (clusters + active - 1) / active;
+        const long long cost = waves * (chunks / k) + 2 * k;  // + a small cost per extra cluster member
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = k;
+        }
+    }
+    return best;
+}
+
 template <int DC, int DR>
 int run_cache_write(const videomla_dims* d, const void* x, int B, int n_tok, const void* W_dkv, const void* W_kr,
                     const float* gamma, void* cache, int slots, int first_slot, unsigned flags, cudaStream_t st) {
@@ -135,9 +183,17 @@ int run_cache_write(const videomla_dims* d, const void* x, int B, int n_tok, con
         const uint32_t box[2] = {64, uint32_t(DR)};
         if (!make_map(&tr, W_kr, 2, dims, str, box, 128)) return VIDEOMLA_ECUDA;
     }
+    auto kern = vmla::cache_write_kernel<DC, DR>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+        return VIDEOMLA_ECUDA;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess)
+        return VIDEOMLA_ECUDA;
+    const int tiles = (n_tok + C::BM - 1) / C::BM;
+    const int ksplit = pick_ksplit(kern, C::THREADS, C::SMEM, d->d_model / C::BKK, tiles * B, C::KS_MAX);
     vmla::CacheWriteParams p;
     p.n_tok = n_tok;
     p.d_model = d->d_model;
+    p.ksplit = ksplit;
     p.T_f = T_f;
     p.slots = slots;
     p.first_slot = first_slot;
@@ -146,11 +202,19 @@ int run_cache_write(const videomla_dims* d, const void* x, int B, int n_tok, con
     p.gamma = gamma;
     p.cache = static_cast<__nv_bfloat16*>(cache);
     p.timeout_ns = g_timeout_ns.load();
-    auto kern = vmla::cache_write_kernel<DC, DR>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
-        return VIDEOMLA_ECUDA;
-    dim3 grid((n_tok + C::BM - 1) / C::BM, B);
-    kern<<<grid, C::THREADS, C::SMEM, st>>>(tx, tw, tr, p);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(tiles, ksplit, B);
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = ksplit;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tx, tw, tr, p) != cudaSuccess) return VIDEOMLA_ECUDA;
     return launch_status(kern, C::SMEM);
 }
 
