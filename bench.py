@@ -151,33 +151,44 @@ class ClockSampler:
                 "power_w_max": max(r[2] for r in rows), "samples": len(loaded), "reasons": reasons}
 
 
-def dist_setup():
+def dist_setup(backend: str = "nccl"):
+    """One process per GPU (torchrun env).  Each rank runs an independent replica
+    of the workload: the process group only carries barriers and the max of the
+    per-rank timings, never data of the hot path."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     return world, rank, local
 
 
-def max_over_ranks(v: float, world: int) -> float:
+def max_over_ranks(v: float, world: int, device: str = "cuda") -> float:
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
-def barrier(world: int):
+def barrier(world: int, cuda: bool = True):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    if cuda:
+        torch.cuda.synchronize()
+
+
+def job_throughput(world: int, units_per_rank: float, ms_max: float, steps: int) -> float:
+    """Whole-job rate: the units every rank processed over the slowest rank's time."""
+    return world * units_per_rank / (ms_max * 1e-3 / steps)
 
 
 # ---------------------------------------------------------------------------
@@ -363,7 +374,7 @@ def run_gpu(args):
         sustained = sm is not None and sm < 1700.0
         peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
         achieved = fl_attn / (attn_ms * 1e-3) / 1e12
-        value = world * fl_step / (ms * 1e-3 / args.steps) / 1e12
+        value = job_throughput(world, fl_step, ms, args.steps) / 1e12
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
@@ -384,11 +395,11 @@ def run_gpu(args):
                          "traffic": ncu_traffic("attention_kernel"),
                          "algorithmic_flops_per_launch": fl_attn},
             "attention_ms": attn_ms, "cache_write_ms": cw_ms,
-            "query_tokens_per_s": wl.n_query * world / (ms * 1e-3 / args.steps),
+            "query_tokens_per_s": job_throughput(world, wl.n_query, ms, args.steps),
             "explicit_mha_equivalent_tflops": flops_explicit_equivalent(d, wl.batch, wl.n_query, Nk)
             / (attn_ms * 1e-3) / 1e12,
             "cache_write_stack": cw_stack,
-            "e2e": {"value": world * fl_step / (e2e_ms * 1e-3 / args.steps) / 1e12, "unit": "TFLOP/s",
+            "e2e": {"value": job_throughput(world, fl_step, e2e_ms, args.steps) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                     "ms_per_step": e2e_ms / args.steps},
             "clocks": clocks,

@@ -199,6 +199,16 @@ int videomla_device_status(int reset);
  */
 uint64_t videomla_set_wait_timeout_ns(uint64_t ns);
 
+/*
+ * Self-test of the failure-detection path: launches one CTA that waits, with the
+ * same bounded wait the kernels use, on a shared-memory barrier that nothing
+ * ever completes.  After ``timeout_ns`` the wait gives up, records
+ * VIDEOMLA_ETIMEOUT in the device status word and the kernel returns normally;
+ * the context stays usable.  Returns the launch status (VIDEOMLA_OK once
+ * enqueued); read the outcome with videomla_device_status().
+ */
+int videomla_selftest_wait_timeout(uint64_t timeout_ns, void* stream);
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 int videomla_version(void);
 

@@ -102,6 +102,19 @@ __device__ __noinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uin
     }
 }
 
+// One CTA waits on a barrier that nothing completes: exercises the bounded wait.
+__global__ void wait_timeout_selftest_kernel(uint64_t timeout_ns) {
+    __shared__ uint64_t bar;
+    __shared__ AbortState ab;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        ab.flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    mbar_wait(&bar, 0, &ab, timeout_ns, 99);  // no arrive ever comes
+}
+
 // ------------------------------------------------------------------------
 // TMA tile loads (no cluster multicast anywhere in this library)
 // ------------------------------------------------------------------------

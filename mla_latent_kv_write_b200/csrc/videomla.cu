@@ -467,6 +467,13 @@ uint64_t videomla_set_wait_timeout_ns(uint64_t ns) {
     return g_timeout_ns.exchange(ns == 0 ? kDefaultTimeoutNs : ns);
 }
 
+int videomla_selftest_wait_timeout(uint64_t timeout_ns, void* stream) {
+    if (timeout_ns == 0 || timeout_ns > 10000000000ull) return VIDEOMLA_EINVAL;
+    if (int rc = check_device()) return rc;
+    vmla::wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns);
+    return cudaGetLastError() == cudaSuccess ? VIDEOMLA_OK : VIDEOMLA_ECUDA;
+}
+
 int videomla_version(void) { return 100; }
 
 }  // extern "C"

@@ -32,6 +32,7 @@ EXPORTED = (
     "videomla_strerror",
     "videomla_device_status",
     "videomla_set_wait_timeout_ns",
+    "videomla_selftest_wait_timeout",
     "videomla_version",
 )
 
@@ -80,6 +81,8 @@ def load_library() -> ctypes.CDLL:
         lib.videomla_device_status.restype = ci
         lib.videomla_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
         lib.videomla_set_wait_timeout_ns.restype = ctypes.c_uint64
+        lib.videomla_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+        lib.videomla_selftest_wait_timeout.restype = ci
         lib.videomla_version.argtypes = []
         lib.videomla_version.restype = ci
         _LIB = lib
