@@ -10,15 +10,19 @@
 //
 // A pre-pass (rope_window_kernel) forms the active window once per call: every
 // valid cached k^R is rotated by its window-local position into an fp16
-// workspace.  Then one CTA per (128-query tile, head, batch element), 192 threads:
+// workspace.  Then one CTA per (128-query tile, head, batch element), 224 threads:
 //   warp 0     TMA producer: q_nope / W_uk (prologue), key tiles (128 keys:
 //              latent from the cache, rotated rope key from the workspace) into
 //              a 4-stage ring, W_uv (epilogue)
-//   warp 1     tcgen05.mma issuer and tensor-memory owner
+//   warp 1     tensor-memory owner; issues the q_abs, S = Q K^T and W_uv MMAs
 //   warps 2-5  softmax: q_abs -> bf16 Q in TMEM, q^R rotation, fp32 online
 //              softmax (row max / sum reduced across the 4 threads of a row
 //              with warp shuffles), P -> TMEM, O rescale, normalisation,
 //              W_uv epilogue and the output stores
+//   warp 6     issues the O += P C MMAs
+// The two MMA streams come from two threads so that S_{j+1} and PV_j are
+// queued to the tensor core independently: neither waits behind the other's
+// dependency.
 // Tensor memory (512 columns, fp32 unless noted):
 //   O [0, d_c)  S [d_c, d_c+128)  P (bf16 pairs) [+128, +64)
 //   Q (bf16 pairs of q_abs, then fp16 pairs of the rotated q^R)
@@ -76,7 +80,7 @@ struct AttnCfg {
     static constexpr int WUV_ATOM = DV * 128, WUV_BYTES = C_ATOMS * WUV_ATOM;
     static constexpr int OLAT_ATOM = BM * 128;
     static constexpr int SMEM = NS * STAGE + 1024 + 1024;
-    static constexpr int THREADS = 192;
+    static constexpr int THREADS = 224;
     static_assert(DC % 64 == 0 && DC <= 256, "latent width");
     static_assert(DR == 16 || DR == 32 || DR == 64, "rope width");
     static_assert(DN % 16 == 0 && DV % 32 == 0 && DV <= 256, "head widths");
@@ -87,7 +91,7 @@ struct AttnCfg {
 
 struct AttnBarriers {
     uint64_t full[4], empty[4];
-    uint64_t q_full, qabs_done, q_ready, s_full, s_free, p_full, pv_done, olat_ready, out_full, drain;
+    uint64_t q_full, qabs_done, q_ready, s_full, s_free, p_full, pv_done, olat_ready, out_full, drain, drain2;
     uint32_t tmem_base;
     AbortState ab;
 };
@@ -150,7 +154,7 @@ __global__ void __launch_bounds__(256) rope_window_kernel(const __nv_bfloat16* _
 }
 
 template <class C>
-__global__ void __launch_bounds__(192, 1) attention_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
+__global__ void __launch_bounds__(224, 1) attention_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     constexpr int DC = C::DC, DR = C::DR, DN = C::DN, DV = C::DV, BM = C::BM, BK = C::BK, NS = C::NS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -179,6 +183,7 @@ __global__ void __launch_bounds__(192, 1) attention_kernel(const __grid_constant
         mbar_init(&bar->olat_ready, 4);
         mbar_init(&bar->out_full, 1);
         mbar_init(&bar->drain, 1);
+        mbar_init(&bar->drain2, 1);
         ab->flag = 0;
         fence_mbar_init();
     }
@@ -256,40 +261,23 @@ __global__ void __launch_bounds__(192, 1) attention_kernel(const __grid_constant
             }
             constexpr uint32_t id_s = idesc_bf16_f32(128, BK, false, false);
             constexpr uint32_t id_s_rope = idesc_f16_f32(128, BK, false, false);
-            constexpr uint32_t id_pv = idesc_bf16_f32(128, DC, false, true);
-            for (int j = 0; ok && j <= nt; ++j) {
-                if (j < nt) {
-                    // S_j = Q . K_j^T : K = DC latent (bf16) + DR rotated rope (fp16) columns
-                    const int s = j % NS;
-                    ok = mbar_wait(&bar->full[s], (j / NS) & 1, ab, to, 32);
-                    if (ok && j > 0) ok = mbar_wait(&bar->s_free, (j - 1) & 1, ab, to, 33);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t st = smem_u32(stage(s));
+            for (int j = 0; ok && j < nt; ++j) {
+                // S_j = Q . K_j^T : K = DC latent (bf16) + DR rotated rope (fp16) columns
+                const int s = j % NS;
+                ok = mbar_wait(&bar->full[s], (j / NS) & 1, ab, to, 32);
+                if (ok && j > 0) ok = mbar_wait(&bar->s_free, (j - 1) & 1, ab, to, 33);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t st = smem_u32(stage(s));
 #pragma unroll
-                    for (int k = 0; k < DC / 16; ++k)
-                        umma_ts(tmem + C::S_COL, tmem + C::Q_COL + k * 8,
-                                sdesc(st + (k / 4) * C::C_ATOM + (k % 4) * 32, 16, 1024, SW128), id_s, k > 0);
+                for (int k = 0; k < DC / 16; ++k)
+                    umma_ts(tmem + C::S_COL, tmem + C::Q_COL + k * 8,
+                            sdesc(st + (k / 4) * C::C_ATOM + (k % 4) * 32, 16, 1024, SW128), id_s, k > 0);
 #pragma unroll
-                    for (int k = 0; k < DR / 16; ++k)
-                        umma_ts(tmem + C::S_COL, tmem + C::Q_COL + DC / 2 + k * 8,
-                                sdesc(st + C::C_ATOMS * C::C_ATOM + k * 32, 16, 8 * C::R_ROWB, C::R_SW), id_s_rope, 1);
-                    umma_commit(&bar->s_full);
-                }
-                if (j > 0) {
-                    // O += P_{j-1} . C_{j-1} : B is the latent block of the same tile, MN-major
-                    const int jj = j - 1, sp = jj % NS;
-                    ok = mbar_wait(&bar->p_full, jj & 1, ab, to, 34);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t st = smem_u32(stage(sp));
-#pragma unroll
-                    for (int k = 0; k < BK / 16; ++k)
-                        umma_ts(tmem + C::O_COL, tmem + C::P_COL + k * 8, sdesc(st + k * 2048, C::C_ATOM, 1024, SW128),
-                                id_pv, (jj > 0 || k > 0));
-                    umma_commit(&bar->empty[sp]);
-                    umma_commit(&bar->pv_done);
-                }
+                for (int k = 0; k < DR / 16; ++k)
+                    umma_ts(tmem + C::S_COL, tmem + C::Q_COL + DC / 2 + k * 8,
+                            sdesc(st + C::C_ATOMS * C::C_ATOM + k * 32, 16, 8 * C::R_ROWB, C::R_SW), id_s_rope, 1);
+                umma_commit(&bar->s_full);
             }
             if (ok) {
                 // out [128 x DV] = (O_hi + O_lo) [128 x DC] . W_uv,h^T  (all K-major SW128):
@@ -315,6 +303,27 @@ __global__ void __launch_bounds__(192, 1) attention_kernel(const __grid_constant
                 umma_commit(&bar->drain);
                 mbar_wait_drain(&bar->drain, 0, to);
             }
+        }
+    } else if (warp == 6) {
+        // ------------------------------------------------------------ PV issuer
+        if (lane == 0) {
+            constexpr uint32_t id_pv = idesc_bf16_f32(128, DC, false, true);
+            bool ok = true;
+            for (int jj = 0; ok && jj < nt; ++jj) {
+                const int sp = jj % NS;
+                ok = mbar_wait(&bar->p_full, jj & 1, ab, to, 34);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t st = smem_u32(stage(sp));
+#pragma unroll
+                for (int k = 0; k < BK / 16; ++k)
+                    umma_ts(tmem + C::O_COL, tmem + C::P_COL + k * 8, sdesc(st + k * 2048, C::C_ATOM, 1024, SW128),
+                            id_pv, (jj > 0 || k > 0));
+                umma_commit(&bar->empty[sp]);
+                umma_commit(&bar->pv_done);
+            }
+            umma_commit(&bar->drain2);
+            mbar_wait_drain(&bar->drain2, 0, to);
         }
     } else {
         // ------------------------------------------------------------ softmax / epilogue

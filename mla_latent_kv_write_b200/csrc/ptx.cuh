@@ -69,13 +69,9 @@ struct AbortState {
     volatile int flag;
 };
 
-// Bounded wait for the phase of ``bar`` with the given parity.  Returns false
-// (without having observed the phase) if the CTA is aborting or the wait ran
-// out of ``timeout_ns``; in the latter case the abort flag and the device
-// status word are set.  ``site`` identifies the wait in the status word.
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, AbortState* ab,
-                                       uint64_t timeout_ns, int site) {
-    if (mbar_try_wait(bar, parity)) return true;
+// Slow path of mbar_wait: the phase was not complete at the first test.
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, AbortState* ab, uint64_t timeout_ns,
+                                            int site) {
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
@@ -89,6 +85,18 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, AbortStat
             }
         }
     }
+}
+
+// Bounded wait for the phase of ``bar`` with the given parity.  Returns false
+// (without having observed the phase) if the CTA is aborting or the wait ran
+// out of ``timeout_ns``; in the latter case the abort flag and the device
+// status word are set.  ``site`` identifies the wait in the status word.
+// The first test is inlined: a call costs the caller its live registers'
+// save and restore, which in the softmax loop is hundreds of cycles.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, AbortState* ab, uint64_t timeout_ns,
+                                          int site) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return mbar_wait_slow(bar, parity, ab, timeout_ns, site);
 }
 
 // Bounded wait used on the unwind path: ignores the abort flag, so that a role
@@ -295,6 +303,13 @@ __device__ __forceinline__ void tmem_st_16x256b_x8(uint32_t taddr, const uint32_
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : VMLA_R8(0), VMLA_R8(8)
+        : "r"(taddr));
+}
+
 // 16 lanes x 128 bit: per repetition k (4 columns), thread i holds
 // r[2k+0] = (lane base + i/4, col 4k + i%4), r[2k+1] = (lane base + i/4 + 8, same col).
 __device__ __forceinline__ void tmem_st_16x128b_x16(uint32_t taddr, const uint32_t (&r)[32]) {
@@ -303,6 +318,18 @@ __device__ __forceinline__ void tmem_st_16x128b_x16(uint32_t taddr, const uint32
         "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
         VMLA_W8(0), VMLA_W8(8), VMLA_W8(16), VMLA_W8(24)
         : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_16x128b_x8(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x128b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        VMLA_W8(0), VMLA_W8(8)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_16x128b_x4(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.16x128b.x4.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), VMLA_W8(0)
+                 : "memory");
 }
 
 #undef VMLA_R8
