@@ -10,19 +10,20 @@
 //
 // A pre-pass (rope_window_kernel) forms the active window once per call: every
 // valid cached k^R is rotated by its window-local position into an fp16
-// workspace.  Then one CTA per (128-query tile, head, batch element), 224 threads:
+// workspace.  Then one CTA per (128-query tile, head, batch element), 352 threads:
 //   warp 0     TMA producer: q_nope / W_uk (prologue), key tiles (128 keys:
 //              latent from the cache, rotated rope key from the workspace) into
 //              a 4-stage ring, W_uv (epilogue)
 //   warp 1     tensor-memory owner; issues the q_abs, S = Q K^T and W_uv MMAs
-//   warps 2-5  softmax: q_abs -> bf16 Q in TMEM, q^R rotation, fp32 online
-//              softmax (row max / sum reduced across the 4 threads of a row
-//              with warp shuffles), P -> TMEM, O rescale, normalisation,
-//              W_uv epilogue and the output stores
-//   warp 6     issues the O += P C MMAs
+//   warps 2-9  softmax, 16 query rows each: q_abs -> bf16 Q in TMEM, q^R
+//              rotation, fp32 online softmax (row max / sum reduced across the
+//              4 threads of a row with warp shuffles), P -> TMEM, O rescale,
+//              normalisation, W_uv epilogue and the output stores
+//   warp 10    issues the O += P C MMAs
 // The two MMA streams come from two threads so that S_{j+1} and PV_j are
 // queued to the tensor core independently: neither waits behind the other's
-// dependency.
+// dependency.  Two softmax warps per SM sub-partition let one warp's exp2 (MUFU)
+// overlap the other's FMA / pack work.
 // Tensor memory (512 columns, fp32 unless noted):
 //   O [0, d_c)  S [d_c, d_c+128)  P (bf16 pairs) [+128, +64)
 //   Q (bf16 pairs of q_abs, then fp16 pairs of the rotated q^R)
@@ -80,7 +81,9 @@ struct AttnCfg {
     static constexpr int WUV_ATOM = DV * 128, WUV_BYTES = C_ATOMS * WUV_ATOM;
     static constexpr int OLAT_ATOM = BM * 128;
     static constexpr int SMEM = NS * STAGE + 1024 + 1024;
-    static constexpr int THREADS = 224;
+    static constexpr int SM_WARPS_PER_HALF = 4;                 // softmax warps per 16-lane half
+    static constexpr int SM_WARPS = 2 * SM_WARPS_PER_HALF;
+    static constexpr int THREADS = 32 * (3 + SM_WARPS);
     static_assert(DC % 64 == 0 && DC <= 256, "latent width");
     static_assert(DR == 16 || DR == 32 || DR == 64, "rope width");
     static_assert(DN % 16 == 0 && DV % 32 == 0 && DV <= 256, "head widths");
@@ -154,7 +157,7 @@ __global__ void __launch_bounds__(256) rope_window_kernel(const __nv_bfloat16* _
 }
 
 template <class C>
-__global__ void __launch_bounds__(224, 1) attention_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
+__global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     constexpr int DC = C::DC, DR = C::DR, DN = C::DN, DV = C::DV, BM = C::BM, BK = C::BK, NS = C::NS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -175,12 +178,12 @@ __global__ void __launch_bounds__(224, 1) attention_kernel(const __grid_constant
         }
         mbar_init(&bar->q_full, 1);
         mbar_init(&bar->qabs_done, 1);
-        mbar_init(&bar->q_ready, 4);
+        mbar_init(&bar->q_ready, C::SM_WARPS);
         mbar_init(&bar->s_full, 1);
-        mbar_init(&bar->s_free, 4);
-        mbar_init(&bar->p_full, 4);
+        mbar_init(&bar->s_free, C::SM_WARPS);
+        mbar_init(&bar->p_full, C::SM_WARPS);
         mbar_init(&bar->pv_done, 1);
-        mbar_init(&bar->olat_ready, 4);
+        mbar_init(&bar->olat_ready, C::SM_WARPS);
         mbar_init(&bar->out_full, 1);
         mbar_init(&bar->drain, 1);
         mbar_init(&bar->drain2, 1);
@@ -304,7 +307,7 @@ __global__ void __launch_bounds__(224, 1) attention_kernel(const __grid_constant
                 mbar_wait_drain(&bar->drain, 0, to);
             }
         }
-    } else if (warp == 6) {
+    } else if (warp == 2 + 2 * C::SM_WARPS_PER_HALF) {
         // ------------------------------------------------------------ PV issuer
         if (lane == 0) {
             constexpr uint32_t id_pv = idesc_bf16_f32(128, DC, false, true);
@@ -325,55 +328,62 @@ __global__ void __launch_bounds__(224, 1) attention_kernel(const __grid_constant
             umma_commit(&bar->drain2);
             mbar_wait_drain(&bar->drain2, 0, to);
         }
-    } else {
+    } else if (warp < 2 + 2 * C::SM_WARPS_PER_HALF) {
         // ------------------------------------------------------------ softmax / epilogue
-        // warps 2-5; a warp may only touch TMEM lanes 32 (warp % 4) .. + 31
+        // warps 2-9.  A warp may only touch TMEM lanes 32 (warp % 4) .. + 31 (its
+        // quadrant); warps 2-5 own lanes 0-15 of their quadrant, warps 6-9 lanes
+        // 16-31, so every query row belongs to exactly one warp and the row max /
+        // sum need no exchange between warps.
         const int w4 = warp & 3;
+        const int half = (warp - 2) >> 2;
         const int quad = lane & 3;
-        const uint32_t tl = tmem + (uint32_t(w4 * 32) << 16);
-        const uint32_t tl16 = tl + (16u << 16);
+        const uint32_t tq = tmem + (uint32_t(w4 * 32) << 16);    // quadrant base (32x32b shapes)
+        const uint32_t tb = tq + (uint32_t(half * 16) << 16);    // this warp's 16 lanes (16xNb shapes)
         const float sl = p.scale_log2;
 
-        // prologue: Q = [bf16(q_abs) | fp16(RoPE3D(q^R))] into TMEM, one row per thread
+        // prologue: Q = [bf16(q_abs) | fp16(RoPE3D(q^R))] into TMEM, one row per
+        // thread; the two warps of a quadrant take alternate 32-column chunks
         bool ok = __all_sync(0xffffffffu, mbar_wait(&bar->qabs_done, 0, ab, to, 40) && !ab->flag);
         if (ok) {
             tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < DC; c += 32) {
+            for (int c = 32 * half; c < DC; c += 64) {
                 uint32_t v[32];
-                tmem_ld_32x32b_x32(tl + C::O_COL + c, v);
+                tmem_ld_32x32b_x32(tq + C::O_COL + c, v);
                 tmem_wait_ld();
                 uint32_t pk[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-                tmem_st_32x32b_x16(tl + C::Q_COL + c / 2, pk);
+                tmem_st_32x32b_x16(tq + C::Q_COL + c / 2, pk);
             }
-            const int r = w4 * 32 + lane;
-            const int i = q0 + r;
-            uint32_t qr[DR / 2];
+            if (half == 0) {
+                const int r = w4 * 32 + lane;
+                const int i = q0 + r;
+                uint32_t qr[DR / 2];
 #pragma unroll
-            for (int e = 0; e < DR / 2; ++e) qr[e] = 0u;
-            if (i < p.Nq) {
-                const uint4* src = reinterpret_cast<const uint4*>(p.q_rope + ((size_t(b) * p.Nq + i) * p.H + h) * DR);
-                const int L = p.q_first + i;
-                const int tq = L / p.T_f;
-                const int pq = L - tq * p.T_f;
-                const int hq = pq / p.grid_w, wq = pq - (pq / p.grid_w) * p.grid_w;
+                for (int e = 0; e < DR / 2; ++e) qr[e] = 0u;
+                if (i < p.Nq) {
+                    const uint4* src = reinterpret_cast<const uint4*>(p.q_rope + ((size_t(b) * p.Nq + i) * p.H + h) * DR);
+                    const int L = p.q_first + i;
+                    const int tq_ = L / p.T_f;
+                    const int pq = L - tq_ * p.T_f;
+                    const int hq = pq / p.grid_w, wq = pq - (pq / p.grid_w) * p.grid_w;
 #pragma unroll
-                for (int c = 0; c < DR / 8; ++c) {
-                    const uint4 v = __ldg(src + c);
-                    qr[4 * c + 0] = rotate_pair(v.x, rope_theta(p, 4 * c + 0, tq, hq, wq));
-                    qr[4 * c + 1] = rotate_pair(v.y, rope_theta(p, 4 * c + 1, tq, hq, wq));
-                    qr[4 * c + 2] = rotate_pair(v.z, rope_theta(p, 4 * c + 2, tq, hq, wq));
-                    qr[4 * c + 3] = rotate_pair(v.w, rope_theta(p, 4 * c + 3, tq, hq, wq));
+                    for (int c = 0; c < DR / 8; ++c) {
+                        const uint4 v = __ldg(src + c);
+                        qr[4 * c + 0] = rotate_pair(v.x, rope_theta(p, 4 * c + 0, tq_, hq, wq));
+                        qr[4 * c + 1] = rotate_pair(v.y, rope_theta(p, 4 * c + 1, tq_, hq, wq));
+                        qr[4 * c + 2] = rotate_pair(v.z, rope_theta(p, 4 * c + 2, tq_, hq, wq));
+                        qr[4 * c + 3] = rotate_pair(v.w, rope_theta(p, 4 * c + 3, tq_, hq, wq));
+                    }
                 }
-            }
-            if constexpr (DR == 16) {
-                tmem_st_32x32b_x8(tl + C::Q_COL + DC / 2, qr);
-            } else if constexpr (DR == 32) {
-                tmem_st_32x32b_x16(tl + C::Q_COL + DC / 2, qr);
-            } else {
-                tmem_st_32x32b_x32(tl + C::Q_COL + DC / 2, qr);
+                if constexpr (DR == 16) {
+                    tmem_st_32x32b_x8(tq + C::Q_COL + DC / 2, qr);
+                } else if constexpr (DR == 32) {
+                    tmem_st_32x32b_x16(tq + C::Q_COL + DC / 2, qr);
+                } else {
+                    tmem_st_32x32b_x32(tq + C::Q_COL + DC / 2, qr);
+                }
             }
             tmem_wait_st();
             tc_fence_before();
@@ -382,23 +392,16 @@ __global__ void __launch_bounds__(224, 1) attention_kernel(const __grid_constant
         }
 
         // main loop.  16x256b layout: this thread holds rows
-        //   R0 = w4*32 + lane/4, R1 = R0 + 8 (lanes 0-15 of the quarter) and
-        //   R2 = R0 + 16, R3 = R0 + 24 (lanes 16-31), 32 columns of each.
-        float m_used[4], l_part[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            m_used[k] = 0.f;
-            l_part[k] = 0.f;
-        }
+        //   R0 = w4*32 + half*16 + lane/4 and R1 = R0 + 8, 32 columns of each
+        //   (columns 8k + 2 quad + {0, 1} of each 64-column half of the tile).
+        float m_used[2] = {0.f, 0.f}, l_part[2] = {0.f, 0.f};
         for (int j = 0; ok && j < nt; ++j) {
             ok = __all_sync(0xffffffffu, mbar_wait(&bar->s_full, j & 1, ab, to, 41));
             if (!ok) break;
             tc_fence_after();
-            uint32_t sa[2][32], sb[2][32];
-            tmem_ld_16x256b_x8(tl + C::S_COL, sa[0]);
-            tmem_ld_16x256b_x8(tl + C::S_COL + 64, sa[1]);
-            tmem_ld_16x256b_x8(tl16 + C::S_COL, sb[0]);
-            tmem_ld_16x256b_x8(tl16 + C::S_COL + 64, sb[1]);
+            uint32_t sv[2][32];
+            tmem_ld_16x256b_x8(tb + C::S_COL, sv[0]);
+            tmem_ld_16x256b_x8(tb + C::S_COL + 64, sv[1]);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
@@ -412,108 +415,84 @@ __global__ void __launch_bounds__(224, 1) attention_kernel(const __grid_constant
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
 #pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int col = 64 * c + 8 * k + 2 * quad + e;
-                            if (col >= valid) {
-                                sa[c][4 * k + e] = sa[c][4 * k + 2 + e] = 0xff800000u;  // -inf
-                                sb[c][4 * k + e] = sb[c][4 * k + 2 + e] = 0xff800000u;
-                            }
-                        }
+                        for (int e = 0; e < 2; ++e)
+                            if (64 * c + 8 * k + 2 * quad + e >= valid)
+                                sv[c][4 * k + e] = sv[c][4 * k + 2 + e] = 0xff800000u;  // -inf
             }
-            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
             for (int c = 0; c < 2; ++c)
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    mx[0] = fmaxf(mx[0], fmaxf(__uint_as_float(sa[c][4 * k]), __uint_as_float(sa[c][4 * k + 1])));
-                    mx[1] = fmaxf(mx[1], fmaxf(__uint_as_float(sa[c][4 * k + 2]), __uint_as_float(sa[c][4 * k + 3])));
-                    mx[2] = fmaxf(mx[2], fmaxf(__uint_as_float(sb[c][4 * k]), __uint_as_float(sb[c][4 * k + 1])));
-                    mx[3] = fmaxf(mx[3], fmaxf(__uint_as_float(sb[c][4 * k + 2]), __uint_as_float(sb[c][4 * k + 3])));
+                    mx[0] = fmaxf(mx[0], fmaxf(__uint_as_float(sv[c][4 * k]), __uint_as_float(sv[c][4 * k + 1])));
+                    mx[1] = fmaxf(mx[1], fmaxf(__uint_as_float(sv[c][4 * k + 2]), __uint_as_float(sv[c][4 * k + 3])));
                 }
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {  // the 4 threads of a row hold its 128 columns
+            for (int k = 0; k < 2; ++k) {  // the 4 threads of a row hold its 128 columns
                 mx[k] = fmaxf(mx[k], __shfl_xor_sync(0xffffffffu, mx[k], 1));
                 mx[k] = fmaxf(mx[k], __shfl_xor_sync(0xffffffffu, mx[k], 2));
             }
             bool waited = false;
             if (j == 0) {
-#pragma unroll
-                for (int k = 0; k < 4; ++k) m_used[k] = mx[k];
+                m_used[0] = mx[0];
+                m_used[1] = mx[1];
             } else {
                 // Rescale only when some row's max grew by more than 2^8 in probability
                 // units; otherwise keep the stale max (exact, p <= 256 fits bf16 / fp32).
-                bool need = false;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) need |= (mx[k] - m_used[k]) * sl > 8.0f;
+                const bool need = (mx[0] - m_used[0]) * sl > 8.0f || (mx[1] - m_used[1]) * sl > 8.0f;
                 if (__any_sync(0xffffffffu, need)) {
                     ok = __all_sync(0xffffffffu, mbar_wait(&bar->pv_done, (j - 1) & 1, ab, to, 42));
                     if (!ok) break;
                     waited = true;
                     tc_fence_after();
-                    float f[4];
+                    float f[2];
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
+                    for (int k = 0; k < 2; ++k) {
                         const float mn = fmaxf(m_used[k], mx[k]);
                         f[k] = ex2((m_used[k] - mn) * sl);
                         m_used[k] = mn;
                         l_part[k] *= f[k];
                     }
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const uint32_t base = half ? tl16 : tl;
-                        const float fa = f[2 * half], fb = f[2 * half + 1];
 #pragma unroll 1
-                        for (int cc = 0; cc < DC; cc += 64) {
-                            uint32_t o[32];
-                            tmem_ld_16x256b_x8(base + C::O_COL + cc, o);
-                            tmem_wait_ld();
+                    for (int cc = 0; cc < DC; cc += 64) {
+                        uint32_t o[32];
+                        tmem_ld_16x256b_x8(tb + C::O_COL + cc, o);
+                        tmem_wait_ld();
 #pragma unroll
-                            for (int k = 0; k < 8; ++k) {
-                                o[4 * k + 0] = __float_as_uint(__uint_as_float(o[4 * k + 0]) * fa);
-                                o[4 * k + 1] = __float_as_uint(__uint_as_float(o[4 * k + 1]) * fa);
-                                o[4 * k + 2] = __float_as_uint(__uint_as_float(o[4 * k + 2]) * fb);
-                                o[4 * k + 3] = __float_as_uint(__uint_as_float(o[4 * k + 3]) * fb);
-                            }
-                            tmem_st_16x256b_x8(base + C::O_COL + cc, o);
+                        for (int k = 0; k < 8; ++k) {
+                            o[4 * k + 0] = __float_as_uint(__uint_as_float(o[4 * k + 0]) * f[0]);
+                            o[4 * k + 1] = __float_as_uint(__uint_as_float(o[4 * k + 1]) * f[0]);
+                            o[4 * k + 2] = __float_as_uint(__uint_as_float(o[4 * k + 2]) * f[1]);
+                            o[4 * k + 3] = __float_as_uint(__uint_as_float(o[4 * k + 3]) * f[1]);
                         }
+                        tmem_st_16x256b_x8(tb + C::O_COL + cc, o);
                     }
                 }
             }
             // P = exp2(s * sl - m * sl), packed bf16 pairs for the 16x128b store:
             // rep kk (4 columns) <- pair (8k + 2 quad, +1) of column half c, kk = 8c + k
-            float nm[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) nm[k] = -m_used[k] * sl;
-            uint32_t pa[32], pb[32];
+            const float nm0 = -m_used[0] * sl, nm1 = -m_used[1] * sl;
+            uint32_t pa[32];
 #pragma unroll
             for (int c = 0; c < 2; ++c)
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const int kk = 8 * c + k;
-                    const float a0 = ex2(fmaf(__uint_as_float(sa[c][4 * k + 0]), sl, nm[0]));
-                    const float a1 = ex2(fmaf(__uint_as_float(sa[c][4 * k + 1]), sl, nm[0]));
-                    const float a2 = ex2(fmaf(__uint_as_float(sa[c][4 * k + 2]), sl, nm[1]));
-                    const float a3 = ex2(fmaf(__uint_as_float(sa[c][4 * k + 3]), sl, nm[1]));
-                    const float b0 = ex2(fmaf(__uint_as_float(sb[c][4 * k + 0]), sl, nm[2]));
-                    const float b1 = ex2(fmaf(__uint_as_float(sb[c][4 * k + 1]), sl, nm[2]));
-                    const float b2 = ex2(fmaf(__uint_as_float(sb[c][4 * k + 2]), sl, nm[3]));
-                    const float b3 = ex2(fmaf(__uint_as_float(sb[c][4 * k + 3]), sl, nm[3]));
+                    const float a0 = ex2(fmaf(__uint_as_float(sv[c][4 * k + 0]), sl, nm0));
+                    const float a1 = ex2(fmaf(__uint_as_float(sv[c][4 * k + 1]), sl, nm0));
+                    const float a2 = ex2(fmaf(__uint_as_float(sv[c][4 * k + 2]), sl, nm1));
+                    const float a3 = ex2(fmaf(__uint_as_float(sv[c][4 * k + 3]), sl, nm1));
                     l_part[0] += a0 + a1;
                     l_part[1] += a2 + a3;
-                    l_part[2] += b0 + b1;
-                    l_part[3] += b2 + b3;
                     pa[2 * kk + 0] = pack_bf16(a0, a1);
                     pa[2 * kk + 1] = pack_bf16(a2, a3);
-                    pb[2 * kk + 0] = pack_bf16(b0, b1);
-                    pb[2 * kk + 1] = pack_bf16(b2, b3);
                 }
             if (j > 0 && !waited) {  // P_{j-1} must have been consumed before P_j overwrites it
                 ok = __all_sync(0xffffffffu, mbar_wait(&bar->pv_done, (j - 1) & 1, ab, to, 43));
                 if (!ok) break;
                 tc_fence_after();
             }
-            tmem_st_16x128b_x16(tl + C::P_COL, pa);
-            tmem_st_16x128b_x16(tl16 + C::P_COL, pb);
+            tmem_st_16x128b_x16(tb + C::P_COL, pa);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -523,9 +502,9 @@ __global__ void __launch_bounds__(224, 1) attention_kernel(const __grid_constant
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar->pv_done, (nt - 1) & 1, ab, to, 44) && !ab->flag);
         if (ok) {
             tc_fence_after();
-            float inv[4], lt[4];
+            float inv[2], lt[2];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
+            for (int k = 0; k < 2; ++k) {
                 lt[k] = l_part[k];
                 lt[k] += __shfl_xor_sync(0xffffffffu, lt[k], 1);
                 lt[k] += __shfl_xor_sync(0xffffffffu, lt[k], 2);
@@ -535,31 +514,26 @@ __global__ void __launch_bounds__(224, 1) attention_kernel(const __grid_constant
             // (nt+1) % NS and (nt+2) % NS (both drained: every PV has completed)
             uint8_t* ol = stage((nt + 1) % NS);
             uint8_t* ol2 = stage((nt + 2) % NS);
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const uint32_t base = half ? tl16 : tl;
-                const int r_top = w4 * 32 + half * 16 + (lane >> 2);
-                const int r_bot = r_top + 8;
-                const float ia = inv[2 * half], ib = inv[2 * half + 1];
+            const int r_top = w4 * 32 + half * 16 + (lane >> 2);
+            const int r_bot = r_top + 8;
 #pragma unroll 1
-                for (int cc = 0; cc < DC / 64; ++cc) {
-                    uint32_t o[32];
-                    tmem_ld_16x256b_x8(base + C::O_COL + cc * 64, o);
-                    tmem_wait_ld();
-                    const int off_top = cc * C::OLAT_ATOM + r_top * 128 + 4 * quad;
-                    const int off_bot = cc * C::OLAT_ATOM + r_bot * 128 + 4 * quad;
+            for (int cc = 0; cc < DC / 64; ++cc) {
+                uint32_t o[32];
+                tmem_ld_16x256b_x8(tb + C::O_COL + cc * 64, o);
+                tmem_wait_ld();
+                const int off_top = cc * C::OLAT_ATOM + r_top * 128 + 4 * quad;
+                const int off_bot = cc * C::OLAT_ATOM + r_bot * 128 + 4 * quad;
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        uint32_t hi, lo;
-                        split_bf16(__uint_as_float(o[4 * k]) * ia, __uint_as_float(o[4 * k + 1]) * ia, hi, lo);
-                        const int ot = off_top + ((k ^ (r_top & 7)) << 4);
-                        *reinterpret_cast<uint32_t*>(ol + ot) = hi;
-                        *reinterpret_cast<uint32_t*>(ol2 + ot) = lo;
-                        split_bf16(__uint_as_float(o[4 * k + 2]) * ib, __uint_as_float(o[4 * k + 3]) * ib, hi, lo);
-                        const int ob = off_bot + ((k ^ (r_bot & 7)) << 4);
-                        *reinterpret_cast<uint32_t*>(ol + ob) = hi;
-                        *reinterpret_cast<uint32_t*>(ol2 + ob) = lo;
-                    }
+                for (int k = 0; k < 8; ++k) {
+                    uint32_t hi, lo;
+                    split_bf16(__uint_as_float(o[4 * k]) * inv[0], __uint_as_float(o[4 * k + 1]) * inv[0], hi, lo);
+                    const int ot = off_top + ((k ^ (r_top & 7)) << 4);
+                    *reinterpret_cast<uint32_t*>(ol + ot) = hi;
+                    *reinterpret_cast<uint32_t*>(ol2 + ot) = lo;
+                    split_bf16(__uint_as_float(o[4 * k + 2]) * inv[1], __uint_as_float(o[4 * k + 3]) * inv[1], hi, lo);
+                    const int ob = off_bot + ((k ^ (r_bot & 7)) << 4);
+                    *reinterpret_cast<uint32_t*>(ol + ob) = hi;
+                    *reinterpret_cast<uint32_t*>(ol2 + ob) = lo;
                 }
             }
             fence_proxy_async_smem();
@@ -569,22 +543,24 @@ __global__ void __launch_bounds__(224, 1) attention_kernel(const __grid_constant
 
             if (p.lse != nullptr && quad == 0) {
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int i = q0 + w4 * 32 + (lane >> 2) + 8 * k;
+                for (int k = 0; k < 2; ++k) {
+                    const int i = q0 + r_top + 8 * k;
                     if (i < p.Nq)
                         p.lse[(size_t(b) * p.Nq + i) * p.H + h] = (m_used[k] * sl + __log2f(lt[k])) * 0.69314718055994531f;
                 }
             }
 
+            // out rows of this quadrant, one per thread; the two warps of a quadrant
+            // take alternate 32-column chunks
             ok = __all_sync(0xffffffffu, mbar_wait(&bar->out_full, 0, ab, to, 45) && !ab->flag);
             if (ok) {
                 tc_fence_after();
                 const int i = q0 + w4 * 32 + lane;
                 __nv_bfloat16* dst = p.out + ((size_t(b) * p.Nq + i) * p.H + h) * DV;
 #pragma unroll 1
-                for (int c = 0; c < DV; c += 32) {
+                for (int c = 32 * half; c < DV; c += 64) {
                     uint32_t v[32];
-                    tmem_ld_32x32b_x32(tl + C::S_COL + c, v);
+                    tmem_ld_32x32b_x32(tq + C::S_COL + c, v);
                     tmem_wait_ld();
                     uint32_t pk[16];
 #pragma unroll
