@@ -59,18 +59,92 @@ struct CacheWriteCfg {
     // rows received from the peers for a K split ks: (ks - 1) * ceil(128 / ks)
     static constexpr int recv_rows(int ks) { return (ks - 1) * ((BM + ks - 1) / ks); }
     static constexpr bool fits(int ks) {
-        return PART_BYTES + recv_rows(ks) * RED_STRIDE * 4 + 1024 + 256 <= SMEM_LIMIT;
+        return PART_BYTES + recv_rows(ks) * RED_STRIDE * 4 + 1024 + 256 + DC * 4 <= SMEM_LIMIT;
     }
     static constexpr int KS_MAX = N > 256 ? 1 : fits(4) ? 4 : fits(3) ? 3 : fits(2) ? 2 : 1;  // cluster size
     static constexpr int RED_BYTES = PART_BYTES + recv_rows(KS_MAX) * RED_STRIDE * 4;
     static constexpr int BUF = NS * STAGE > RED_BYTES ? NS * STAGE : RED_BYTES;
-    static constexpr int SMEM = BUF + 1024 + 256;
+    static constexpr int SMEM = BUF + 1024 + 256 + DC * 4;  // stages | barriers | gamma
     static_assert(SMEM <= SMEM_LIMIT, "shared memory");
     static constexpr int THREADS = 192;
     static_assert(N % 16 == 0 && N_CHUNK % 16 == 0 && N_CHUNK <= 256, "MMA N");
     static_assert(DC % 32 == 0 && DR % 16 == 0 && DC % WBOX == 0, "widths");
     static_assert(N % 8 == 0 && N / 8 <= 64 && DC % 8 == 0, "a warp covers a row in 8-column groups");
 };
+
+// Rows [r_lo, r_hi) of this CTA's tile: sum the KS partials (this CTA's in
+// ``part``, the peers' in the ``rbuf`` slots), RMSNorm of the latent columns with
+// the gain ``gs``, bf16 rows into the ring slot of their frame.  Four threads per
+// row (a quad of lanes); thread q of the quad holds the 8-column groups q, q + 4,
+// ... so that each step of the quad covers 128 contiguous bytes; the row's sum of
+// squares is reduced over the quad with warp shuffles.  KS is a template argument
+// so that every partial of a group is loaded before any is summed.
+template <int DC, int DR, int KS>
+__device__ __forceinline__ void cw_finish_rows(const CacheWriteParams& p, const float* part, const float* rbuf,
+                                               const float* gs, int rows_max, int r_lo, int r_hi, int row0, int b,
+                                               bool store) {
+    using C = CacheWriteCfg<DC, DR>;
+    constexpr int N = C::N, GROUPS = N / 8, GPT = (GROUPS + 3) / 4;
+    const int q = threadIdx.x & 3;
+    for (int r0 = r_lo; r0 < r_hi; r0 += C::THREADS / 4) {  // warp-uniform trip count
+        const int r = r0 + int(threadIdx.x >> 2);
+        const int token = row0 + r;
+        const bool live = store && r < r_hi && token < p.n_tok;
+        float a[GPT][8];
+#pragma unroll
+        for (int i = 0; i < GPT; ++i) {
+            const int grp = q + 4 * i;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) a[i][e] = 0.f;
+            if (live && grp < GROUPS) {
+                float4 u[KS][2];
+#pragma unroll
+                for (int k = 0; k < KS; ++k) {
+                    const float* src = k == 0 ? part + r * C::RED_STRIDE + 8 * grp
+                                              : rbuf + ((k - 1) * rows_max + (r - r_lo)) * C::RED_STRIDE + 8 * grp;
+                    u[k][0] = *reinterpret_cast<const float4*>(src);
+                    u[k][1] = *reinterpret_cast<const float4*>(src + 4);
+                }
+#pragma unroll
+                for (int k = 0; k < KS; ++k) {
+                    a[i][0] += u[k][0].x; a[i][1] += u[k][0].y; a[i][2] += u[k][0].z; a[i][3] += u[k][0].w;
+                    a[i][4] += u[k][1].x; a[i][5] += u[k][1].y; a[i][6] += u[k][1].z; a[i][7] += u[k][1].w;
+                }
+            }
+        }
+        float scale = 1.0f;
+        if (p.normalize) {
+            float ss = 0.f;
+#pragma unroll
+            for (int i = 0; i < GPT; ++i)
+                if (q + 4 * i < DC / 8) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) ss = fmaf(a[i][e], a[i][e], ss);
+                }
+            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+            ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+            scale = rsqrtf(ss * (1.0f / DC) + p.eps);
+        }
+        if (live) {
+            const int frame = token / p.T_f;
+            const int slot = (p.first_slot + frame) % p.slots;
+            const long long row = (long long)b * p.slots * p.T_f + (long long)slot * p.T_f + (token - frame * p.T_f);
+            uint4* out = reinterpret_cast<uint4*>(p.cache + row * N);
+#pragma unroll
+            for (int i = 0; i < GPT; ++i) {
+                const int grp = q + 4 * i;
+                if (grp < GROUPS) {
+                    const bool norm = p.normalize && grp < DC / 8;
+                    float o[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) o[e] = norm ? a[i][e] * scale * gs[8 * grp + e] : a[i][e];
+                    out[grp] = make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]),
+                                          pack_bf16(o[6], o[7]));
+                }
+            }
+        }
+    }
+}
 
 template <int DC, int DR>
 __global__ void __launch_bounds__(192, 1)
@@ -89,6 +163,7 @@ __global__ void __launch_bounds__(192, 1)
     AbortState* ab = reinterpret_cast<AbortState*>(tmem_slot + 1);
     float* part = reinterpret_cast<float*>(smem);  // fp32 partial [BM][RED_STRIDE], reuses the stages
     float* rbuf = reinterpret_cast<float*>(smem + C::PART_BYTES);  // [ks-1][rows_max][RED_STRIDE]
+    float* gs = reinterpret_cast<float*>(smem + C::BUF + 256);      // RMSNorm gain [DC]
 
     const int warp = warp_id(), lane = lane_id();
     const int row0 = blockIdx.x * C::BM;
@@ -111,6 +186,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         fence_mbar_init();
     }
+    for (int c = threadIdx.x; c < DC; c += C::THREADS) gs[c] = p.gamma != nullptr ? __ldg(p.gamma + c) : 1.0f;
     if (warp == 1) {
         tmem_alloc(tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
@@ -216,7 +292,10 @@ __global__ void __launch_bounds__(192, 1)
             }
         }
         fence_proxy_async_smem();  // the bulk copies read part through the async proxy
-        named_barrier_sync(1, 128);
+    }
+    // every thread of the CTA: all of ``part`` is written before anyone reads or ships it
+    __syncthreads();
+    if (warp >= 2) {
         // (b) ship each peer the contiguous block of its rows: one bulk copy per peer
         if (warp == 2 && lane == 0 && p.ksplit > 1) {
             for (int k = 0; k < p.ksplit; ++k) {
@@ -229,84 +308,20 @@ __global__ void __launch_bounds__(192, 1)
             }
             bulk_commit();
         }
-        // our outgoing copies must have read ``part`` before this CTA exits
-        if (warp == 2 && lane == 0 && p.ksplit > 1) bulk_wait_read();
     }
 
-    // (c) all 192 threads: sum the ksplit partials of this CTA's rows, RMSNorm,
-    // bf16 rows.  Four threads per row (a quad of lanes); thread q of the quad
-    // holds the 8-column groups q, q + 4, ... so that each step of the quad
-    // covers 128 contiguous bytes.  The row's sum of squares is reduced over the
-    // quad with warp shuffles.
+    // (c) all 192 threads: sum the ksplit partials of this CTA's rows, RMSNorm, bf16 rows
     const bool got = p.ksplit == 1 || __all_sync(0xffffffffu, mbar_wait(recv, 0, ab, p.timeout_ns, 4));
     const int r_lo = (C::BM * int(rank)) / p.ksplit, r_hi = (C::BM * (int(rank) + 1)) / p.ksplit;
-    const int q = threadIdx.x & 3;
-    constexpr int GPT = (GROUPS + 3) / 4;  // groups per thread
-    float g[GPT][8];
-#pragma unroll
-    for (int i = 0; i < GPT; ++i)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const int col = 8 * (q + 4 * i) + e;
-            g[i][e] = (p.gamma != nullptr && col < DC) ? __ldg(p.gamma + col) : 1.0f;
-        }
     const bool store = got && !any_abort && !ab->flag;
-    for (int r0 = r_lo; r0 < r_hi; r0 += C::THREADS / 4) {  // warp-uniform trip count
-        const int r = r0 + int(threadIdx.x >> 2);
-        const int token = row0 + r;
-        const bool live = store && r < r_hi && token < p.n_tok;
-        float a[GPT][8];
-#pragma unroll
-        for (int i = 0; i < GPT; ++i) {
-            const int grp = q + 4 * i;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) a[i][e] = 0.f;
-            if (live && grp < GROUPS) {
-                const float* src = part + r * C::RED_STRIDE + 8 * grp;
-                float4 u = *reinterpret_cast<const float4*>(src), w = *reinterpret_cast<const float4*>(src + 4);
-                a[i][0] = u.x; a[i][1] = u.y; a[i][2] = u.z; a[i][3] = u.w;
-                a[i][4] = w.x; a[i][5] = w.y; a[i][6] = w.z; a[i][7] = w.w;
-                for (int sl = 0; sl + 1 < p.ksplit; ++sl) {
-                    const float* sk = rbuf + (sl * rows_max + (r - r_lo)) * C::RED_STRIDE + 8 * grp;
-                    u = *reinterpret_cast<const float4*>(sk);
-                    w = *reinterpret_cast<const float4*>(sk + 4);
-                    a[i][0] += u.x; a[i][1] += u.y; a[i][2] += u.z; a[i][3] += u.w;
-                    a[i][4] += w.x; a[i][5] += w.y; a[i][6] += w.z; a[i][7] += w.w;
-                }
-            }
-        }
-        float scale = 1.0f;
-        if (p.normalize) {
-            float ss = 0.f;
-#pragma unroll
-            for (int i = 0; i < GPT; ++i)
-                if (q + 4 * i < DC / 8) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) ss = fmaf(a[i][e], a[i][e], ss);
-                }
-            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-            ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-            scale = rsqrtf(ss * (1.0f / DC) + p.eps);
-        }
-        if (live) {
-            const int frame = token / p.T_f;
-            const int slot = (p.first_slot + frame) % p.slots;
-            const long long row = (long long)b * p.slots * p.T_f + (long long)slot * p.T_f + (token - frame * p.T_f);
-            uint4* out = reinterpret_cast<uint4*>(p.cache + row * N);
-#pragma unroll
-            for (int i = 0; i < GPT; ++i) {
-                const int grp = q + 4 * i;
-                if (grp < GROUPS) {
-                    const bool norm = p.normalize && grp < DC / 8;
-                    float o[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) o[e] = norm ? a[i][e] * scale * g[i][e] : a[i][e];
-                    out[grp] = make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]),
-                                          pack_bf16(o[6], o[7]));
-                }
-            }
-        }
+    switch (p.ksplit) {
+        case 1: cw_finish_rows<DC, DR, 1>(p, part, rbuf, gs, rows_max, r_lo, r_hi, row0, b, store); break;
+        case 2: cw_finish_rows<DC, DR, 2>(p, part, rbuf, gs, rows_max, r_lo, r_hi, row0, b, store); break;
+        case 3: cw_finish_rows<DC, DR, 3>(p, part, rbuf, gs, rows_max, r_lo, r_hi, row0, b, store); break;
+        default: cw_finish_rows<DC, DR, 4>(p, part, rbuf, gs, rows_max, r_lo, r_hi, row0, b, store); break;
     }
+    // our outgoing copies must have read ``part`` before this CTA exits
+    if (warp == 2 && lane == 0 && p.ksplit > 1) bulk_wait_read();
 
     tc_fence_before();
     __syncthreads();
