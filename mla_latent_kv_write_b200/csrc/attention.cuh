@@ -66,30 +66,51 @@ template <int DC_, int DR_, int DN_, int DV_>
 struct AttnCfg {
     static constexpr int DC = DC_, DR = DR_, DN = DN_, DV = DV_;
     static constexpr int W = DC + DR;  // cached scalars per token
-    static constexpr int BM = 128, BK = 128;
-    static constexpr int C_ATOMS = DC / 64;
-    static constexpr int C_ATOM = BK * 128;           // one 64-column block of the key tile
-    static constexpr int R_ROWB = DR * 2;             // bytes of rotated k^R per key (fp16)
+    static constexpr int BM = 128;
+    // Q (bf16 pairs) stays in tensor memory next to O, S and P when all four fit
+    // in its 512 columns with 128-key tiles; otherwise Q moves to shared memory
+    // (the score MMAs read both operands from there) and key tiles shrink to 64.
+    static constexpr bool QS = DC + 128 + 64 + W / 2 > 512;
+    static constexpr int BK = QS ? 64 : 128;
+    static constexpr int C_ATOMS = (DC + 63) / 64;       // 64-column blocks (the last may be half used)
+    static constexpr int C_ATOM = BK * 128;              // one 64-column block of the key tile
+    static constexpr int R_ROWB = DR * 2;                // bytes of rotated k^R per key (fp16)
     static constexpr uint32_t R_SW = DR == 16 ? SW32 : DR == 32 ? SW64 : SW128;
     static constexpr int STAGE = C_ATOMS * C_ATOM + BK * R_ROWB;
-    static constexpr int NS = (4 * STAGE + 2048 <= 232448) ? 4 : 3;  // pipeline stages
-    static constexpr int O_COL = 0, S_COL = DC, P_COL = DC + BK, Q_COL = DC + BK + BK / 2;
-    static constexpr int TMEM_END = Q_COL + W / 2;
     static constexpr int QN_CHUNKS = DN / 16;
     static constexpr int QN_BYTES = QN_CHUNKS * BM * 32;
     static constexpr int WUK_ATOM = DN * 128, WUK_BYTES = C_ATOMS * WUK_ATOM;
     static constexpr int WUV_ATOM = DV * 128, WUV_BYTES = C_ATOMS * WUV_ATOM;
     static constexpr int OLAT_ATOM = BM * 128;
-    static constexpr int SMEM = NS * STAGE + 1024 + 1024;
+    // Q region (QS only): q_nope and W_uk for the prologue, then Q (bf16 q_abs in
+    // 64-column K-major blocks, fp16 rotated q^R after them), then O_lat
+    static constexpr int Q_ATOM = BM * 128;
+    static constexpr int QR_OFF = C_ATOMS * Q_ATOM;
+    static constexpr int WUK_OFF = (QN_BYTES + 1023) / 1024 * 1024;
+    static constexpr int QBYTES = QS ? QR_OFF + BM * R_ROWB : 0;
+    static constexpr int NS = (4 * STAGE + QBYTES + 2048 <= 232448) ? 4
+                            : (3 * STAGE + QBYTES + 2048 <= 232448) ? 3 : 2;  // key-tile ring stages
+    // W_uv (epilogue) spreads over consecutive ring stages, APS 64-column blocks each
+    static constexpr int APS = STAGE / WUV_ATOM;
+    static constexpr int WUV_STAGES = (C_ATOMS + APS - 1) / APS;
+    // MMAs of N = DC (q_abs, P C) run as NMMA column halves of NCH <= 256
+    static constexpr int NMMA = DC > 256 ? 2 : 1;
+    static constexpr int NCH = DC / NMMA;
+    static constexpr int O_COL = 0, S_COL = DC, P_COL = DC + BK, Q_COL = DC + BK + BK / 2;
+    static constexpr int TMEM_END = QS ? P_COL + BK / 2 : Q_COL + W / 2;
+    static constexpr int SMEM = NS * STAGE + QBYTES + 1024 + 1024;
     static constexpr int SM_WARPS_PER_HALF = 4;                 // softmax warps per 16-lane half
     static constexpr int SM_WARPS = 2 * SM_WARPS_PER_HALF;
     static constexpr int THREADS = 32 * (3 + SM_WARPS);
-    static_assert(DC % 64 == 0 && DC <= 256, "latent width");
+    static_assert(DC % 32 == 0 && NCH % 64 == 0 || NMMA == 1, "latent width");
+    static_assert(DC % 32 == 0 && NCH <= 256, "latent width");
     static_assert(DR == 16 || DR == 32 || DR == 64, "rope width");
     static_assert(DN % 16 == 0 && DV % 32 == 0 && DV <= 256, "head widths");
-    static_assert(TMEM_END <= 512, "tensor memory budget");
-    static_assert(QN_BYTES <= STAGE && WUK_BYTES <= STAGE && WUV_BYTES <= STAGE &&
-                  C_ATOMS * OLAT_ATOM <= STAGE, "prologue / epilogue buffers reuse pipeline stages");
+    static_assert(TMEM_END <= 512 && S_COL + DV <= 512, "tensor memory budget");
+    static_assert(SMEM <= 232448 && APS >= 1, "shared memory budget");
+    static_assert(QS ? (WUK_OFF + WUK_BYTES <= QBYTES && C_ATOMS * OLAT_ATOM <= QBYTES)
+                     : (QN_BYTES <= STAGE && WUK_BYTES <= STAGE && WUV_STAGES == 1 && C_ATOMS * OLAT_ATOM <= STAGE),
+                  "prologue / epilogue buffers reuse the Q region or pipeline stages");
 };
 
 struct AttnBarriers {
@@ -161,7 +182,8 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
     constexpr int DC = C::DC, DR = C::DR, DN = C::DN, DV = C::DV, BM = C::BM, BK = C::BK, NS = C::NS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    AttnBarriers* bar = reinterpret_cast<AttnBarriers*>(smem + NS * C::STAGE);
+    uint8_t* qreg = smem + NS * C::STAGE;  // Q region (QS only)
+    AttnBarriers* bar = reinterpret_cast<AttnBarriers*>(qreg + C::QBYTES);
     AbortState* ab = &bar->ab;
     auto stage = [&](int s) { return smem + s * C::STAGE; };
 
@@ -210,18 +232,20 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
             tma_prefetch_desc(&maps.wuk);
             tma_prefetch_desc(&maps.wuv);
             mbar_arrive_expect_tx(&bar->q_full, C::QN_BYTES + C::WUK_BYTES);
+            uint8_t* qn_dst = C::QS ? qreg : stage(NS - 2);
+            uint8_t* wuk_dst = C::QS ? qreg + C::WUK_OFF : stage(NS - 1);
             for (int c = 0; c < C::QN_CHUNKS; ++c)
-                tma_load_4d(stage(NS - 2) + c * BM * 32, &maps.qn, &bar->q_full, c * 16, h, q0, b);
+                tma_load_4d(qn_dst + c * BM * 32, &maps.qn, &bar->q_full, c * 16, h, q0, b);
             for (int a = 0; a < C::C_ATOMS; ++a)
-                tma_load_2d(stage(NS - 1) + a * C::WUK_ATOM, &maps.wuk, &bar->q_full, a * 64, h * DN);
+                tma_load_2d(wuk_dst + a * C::WUK_ATOM, &maps.wuk, &bar->q_full, a * 64, h * DN);
             int issued = 0;
             bool qabs_seen = false;
-            for (int j = 0; j <= nt; ++j) {
+            for (int j = 0; j < nt + C::WUV_STAGES; ++j) {
                 const int s = j % NS;
                 bool ok = true;
                 if (j >= NS) {
                     ok = mbar_wait(&bar->empty[s], ((j / NS) - 1) & 1, ab, to, 10);
-                } else if (s >= NS - 2 && !qabs_seen) {  // stage still holds q_nope / W_uk
+                } else if (!C::QS && s >= NS - 2 && !qabs_seen) {  // stage still holds q_nope / W_uk
                     ok = qabs_seen = mbar_wait(&bar->qabs_done, 0, ab, to, 11);
                 }
                 if (!ok) break;
@@ -232,10 +256,12 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                     for (int a = 0; a < C::C_ATOMS; ++a)
                         tma_load_3d(stage(s) + a * C::C_ATOM, &maps.cc[run], &bar->full[s], a * 64, row, b);
                     tma_load_3d(stage(s) + C::C_ATOMS * C::C_ATOM, &maps.kr[run], &bar->full[s], 0, row, b);
-                } else {
-                    mbar_arrive_expect_tx(&bar->full[s], C::WUV_BYTES);
-                    for (int a = 0; a < C::C_ATOMS; ++a)
-                        tma_load_2d(stage(s) + a * C::WUV_ATOM, &maps.wuv, &bar->full[s], a * 64, h * DV);
+                } else {  // W_uv blocks [a0, a1) of the epilogue
+                    const int a0 = (j - nt) * C::APS;
+                    const int a1 = a0 + C::APS < C::C_ATOMS ? a0 + C::APS : C::C_ATOMS;
+                    mbar_arrive_expect_tx(&bar->full[s], (a1 - a0) * C::WUV_ATOM);
+                    for (int a = a0; a < a1; ++a)
+                        tma_load_2d(stage(s) + (a - a0) * C::WUV_ATOM, &maps.wuv, &bar->full[s], a * 64, h * DV);
                 }
                 issued = j + 1;
             }
@@ -253,12 +279,16 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                 tc_fence_after();
                 // q_abs [128 x DC] = q_nope [128 x DN] . W_uk,h [DN x DC]   (A: K-major SW32 chunks,
                 // B: MN-major SW128 blocks of 64 latent columns)
-                constexpr uint32_t id_qabs = idesc_bf16_f32(128, DC, false, true);
-                const uint32_t sq = smem_u32(stage(NS - 2)), sw = smem_u32(stage(NS - 1));
+                constexpr uint32_t id_qabs = idesc_bf16_f32(128, C::NCH, false, true);
+                const uint32_t sq = smem_u32(C::QS ? qreg : stage(NS - 2));
+                const uint32_t sw = smem_u32(C::QS ? qreg + C::WUK_OFF : stage(NS - 1));
 #pragma unroll
                 for (int k = 0; k < C::QN_CHUNKS; ++k)
-                    umma_ss(tmem + C::O_COL, sdesc(sq + k * BM * 32, 16, 256, SW32),
-                            sdesc(sw + k * 2048, C::WUK_ATOM, 1024, SW128), id_qabs, k > 0);
+#pragma unroll
+                    for (int n = 0; n < C::NMMA; ++n)
+                        umma_ss(tmem + C::O_COL + n * C::NCH, sdesc(sq + k * BM * 32, 16, 256, SW32),
+                                sdesc(sw + n * (C::NCH / 64) * C::WUK_ATOM + k * 2048, C::WUK_ATOM, 1024, SW128),
+                                id_qabs, k > 0);
                 umma_commit(&bar->qabs_done);
                 ok = mbar_wait(&bar->q_ready, 0, ab, to, 31);
             }
@@ -272,32 +302,49 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t st = smem_u32(stage(s));
+                if constexpr (C::QS) {
+                    const uint32_t sq = smem_u32(qreg);
 #pragma unroll
-                for (int k = 0; k < DC / 16; ++k)
-                    umma_ts(tmem + C::S_COL, tmem + C::Q_COL + k * 8,
-                            sdesc(st + (k / 4) * C::C_ATOM + (k % 4) * 32, 16, 1024, SW128), id_s, k > 0);
+                    for (int k = 0; k < DC / 16; ++k)
+                        umma_ss(tmem + C::S_COL, sdesc(sq + (k / 4) * C::Q_ATOM + (k % 4) * 32, 16, 1024, SW128),
+                                sdesc(st + (k / 4) * C::C_ATOM + (k % 4) * 32, 16, 1024, SW128), id_s, k > 0);
 #pragma unroll
-                for (int k = 0; k < DR / 16; ++k)
-                    umma_ts(tmem + C::S_COL, tmem + C::Q_COL + DC / 2 + k * 8,
-                            sdesc(st + C::C_ATOMS * C::C_ATOM + k * 32, 16, 8 * C::R_ROWB, C::R_SW), id_s_rope, 1);
+                    for (int k = 0; k < DR / 16; ++k)
+                        umma_ss(tmem + C::S_COL, sdesc(sq + C::QR_OFF + k * 32, 16, 8 * C::R_ROWB, C::R_SW),
+                                sdesc(st + C::C_ATOMS * C::C_ATOM + k * 32, 16, 8 * C::R_ROWB, C::R_SW), id_s_rope, 1);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < DC / 16; ++k)
+                        umma_ts(tmem + C::S_COL, tmem + C::Q_COL + k * 8,
+                                sdesc(st + (k / 4) * C::C_ATOM + (k % 4) * 32, 16, 1024, SW128), id_s, k > 0);
+#pragma unroll
+                    for (int k = 0; k < DR / 16; ++k)
+                        umma_ts(tmem + C::S_COL, tmem + C::Q_COL + DC / 2 + k * 8,
+                                sdesc(st + C::C_ATOMS * C::C_ATOM + k * 32, 16, 8 * C::R_ROWB, C::R_SW), id_s_rope, 1);
+                }
                 umma_commit(&bar->s_full);
             }
             if (ok) {
-                // out [128 x DV] = (O_hi + O_lo) [128 x DC] . W_uv,h^T  (all K-major SW128):
-                // O / l is split into two bf16 parts so that its rounding stays ~2^-16
-                const int sw_ = nt % NS, so = (nt + 1) % NS, so2 = (nt + 2) % NS;
-                ok = mbar_wait(&bar->full[sw_], (nt / NS) & 1, ab, to, 35) &&
-                     mbar_wait(&bar->olat_ready, 0, ab, to, 36);
+                // out [128 x DV] = O_lat [128 x DC] . W_uv,h^T  (all K-major SW128).  With Q in
+                // tensor memory, O / l is split into two bf16 parts (hi in stage nt+1, lo in
+                // stage nt+2) so that its rounding stays ~2^-16; with Q in shared memory the
+                // single bf16 part lives in the Q region.  W_uv block a is in stage nt + a / APS.
+                for (int w = 0; ok && w < C::WUV_STAGES; ++w)
+                    ok = mbar_wait(&bar->full[(nt + w) % NS], ((nt + w) / NS) & 1, ab, to, 35);
+                ok = ok && mbar_wait(&bar->olat_ready, 0, ab, to, 36);
                 if (ok) {
                     tc_fence_after();
                     constexpr uint32_t id_o = idesc_bf16_f32(128, DV, false, false);
-                    const uint32_t ao = smem_u32(stage(so)), ao2 = smem_u32(stage(so2)), bw = smem_u32(stage(sw_));
+                    const uint32_t ao = smem_u32(C::QS ? qreg : stage((nt + 1) % NS));
+                    const uint32_t ao2 = smem_u32(stage((nt + 2) % NS));
 #pragma unroll
                     for (int k = 0; k < DC / 16; ++k) {
-                        const uint64_t bd = sdesc(bw + (k / 4) * C::WUV_ATOM + (k % 4) * 32, 16, 1024, SW128);
-                        const uint32_t off = (k / 4) * C::OLAT_ATOM + (k % 4) * 32;
+                        const int a = k / 4;
+                        const uint32_t bw = smem_u32(stage((nt + a / C::APS) % NS)) + (a % C::APS) * C::WUV_ATOM;
+                        const uint64_t bd = sdesc(bw + (k % 4) * 32, 16, 1024, SW128);
+                        const uint32_t off = a * C::OLAT_ATOM + (k % 4) * 32;
                         umma_ss(tmem + C::S_COL, sdesc(ao + off, 16, 1024, SW128), bd, id_o, k > 0);
-                        umma_ss(tmem + C::S_COL, sdesc(ao2 + off, 16, 1024, SW128), bd, id_o, 1);
+                        if constexpr (!C::QS) umma_ss(tmem + C::S_COL, sdesc(ao2 + off, 16, 1024, SW128), bd, id_o, 1);
                     }
                     umma_commit(&bar->out_full);
                 }
@@ -310,7 +357,7 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
     } else if (warp == 2 + 2 * C::SM_WARPS_PER_HALF) {
         // ------------------------------------------------------------ PV issuer
         if (lane == 0) {
-            constexpr uint32_t id_pv = idesc_bf16_f32(128, DC, false, true);
+            constexpr uint32_t id_pv = idesc_bf16_f32(128, C::NCH, false, true);
             bool ok = true;
             for (int jj = 0; ok && jj < nt; ++jj) {
                 const int sp = jj % NS;
@@ -320,8 +367,11 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                 const uint32_t st = smem_u32(stage(sp));
 #pragma unroll
                 for (int k = 0; k < BK / 16; ++k)
-                    umma_ts(tmem + C::O_COL, tmem + C::P_COL + k * 8, sdesc(st + k * 2048, C::C_ATOM, 1024, SW128),
-                            id_pv, (jj > 0 || k > 0));
+#pragma unroll
+                    for (int n = 0; n < C::NMMA; ++n)
+                        umma_ts(tmem + C::O_COL + n * C::NCH, tmem + C::P_COL + k * 8,
+                                sdesc(st + n * (C::NCH / 64) * C::C_ATOM + k * 2048, C::C_ATOM, 1024, SW128), id_pv,
+                                (jj > 0 || k > 0));
                 umma_commit(&bar->empty[sp]);
                 umma_commit(&bar->pv_done);
             }
@@ -341,11 +391,14 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
         const uint32_t tb = tq + (uint32_t(half * 16) << 16);    // this warp's 16 lanes (16xNb shapes)
         const float sl = p.scale_log2;
 
-        // prologue: Q = [bf16(q_abs) | fp16(RoPE3D(q^R))] into TMEM, one row per
-        // thread; the two warps of a quadrant take alternate 32-column chunks
+        // prologue: Q = [bf16(q_abs) | fp16(RoPE3D(q^R))], one row per thread, into
+        // TMEM or (QS) into the Q region of shared memory in the swizzled K-major
+        // layout the score MMAs read; the two warps of a quadrant take alternate
+        // 32-column chunks of q_abs
         bool ok = __all_sync(0xffffffffu, mbar_wait(&bar->qabs_done, 0, ab, to, 40) && !ab->flag);
         if (ok) {
             tc_fence_after();
+            const int r = w4 * 32 + lane;
 #pragma unroll 1
             for (int c = 32 * half; c < DC; c += 64) {
                 uint32_t v[32];
@@ -354,10 +407,18 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                 uint32_t pk[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-                tmem_st_32x32b_x16(tq + C::Q_COL + c / 2, pk);
+                if constexpr (C::QS) {
+                    uint8_t* row_base = qreg + (c / 64) * C::Q_ATOM + r * 128;
+                    const int kc0 = (c % 64) / 8;  // first 16-byte chunk of these 32 columns
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        *reinterpret_cast<uint4*>(row_base + (((kc0 + i) ^ (r & 7)) << 4)) =
+                            make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                } else {
+                    tmem_st_32x32b_x16(tq + C::Q_COL + c / 2, pk);
+                }
             }
             if (half == 0) {
-                const int r = w4 * 32 + lane;
                 const int i = q0 + r;
                 uint32_t qr[DR / 2];
 #pragma unroll
@@ -377,7 +438,18 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                         qr[4 * c + 3] = rotate_pair(v.w, rope_theta(p, 4 * c + 3, tq_, hq, wq));
                     }
                 }
-                if constexpr (DR == 16) {
+                if constexpr (C::QS) {
+                    // rows of R_ROWB bytes with the 16-byte chunk index XOR-ed by address
+                    // bits [7, 7 + log2(R_ROWB / 16)): the 32B / 64B / 128B swizzles
+                    uint8_t* row_base = qreg + C::QR_OFF + r * C::R_ROWB;
+                    constexpr int NCH16 = C::R_ROWB / 16;
+#pragma unroll
+                    for (int e = 0; e < NCH16; ++e) {
+                        const int sw = ((r * C::R_ROWB) >> 7) & (NCH16 - 1);
+                        *reinterpret_cast<uint4*>(row_base + ((e ^ sw) << 4)) =
+                            make_uint4(qr[4 * e], qr[4 * e + 1], qr[4 * e + 2], qr[4 * e + 3]);
+                    }
+                } else if constexpr (DR == 16) {
                     tmem_st_32x32b_x8(tq + C::Q_COL + DC / 2, qr);
                 } else if constexpr (DR == 32) {
                     tmem_st_32x32b_x16(tq + C::Q_COL + DC / 2, qr);
@@ -385,7 +457,8 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                     tmem_st_32x32b_x32(tq + C::Q_COL + DC / 2, qr);
                 }
             }
-            tmem_wait_st();
+            if constexpr (C::QS) fence_proxy_async_smem();  // generic stores -> MMA operand reads
+            else tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar->q_ready);
@@ -399,9 +472,10 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
             ok = __all_sync(0xffffffffu, mbar_wait(&bar->s_full, j & 1, ab, to, 41));
             if (!ok) break;
             tc_fence_after();
-            uint32_t sv[2][32];
-            tmem_ld_16x256b_x8(tb + C::S_COL, sv[0]);
-            tmem_ld_16x256b_x8(tb + C::S_COL + 64, sv[1]);
+            constexpr int NC = BK / 64;  // 64-column halves of the tile
+            uint32_t sv[NC][32];
+#pragma unroll
+            for (int c = 0; c < NC; ++c) tmem_ld_16x256b_x8(tb + C::S_COL + 64 * c, sv[c]);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
@@ -411,7 +485,7 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
             key_tile<BK>(p, j, run, row, valid);
             if (valid < BK) {  // ragged last tile of a run: mask the missing keys
 #pragma unroll
-                for (int c = 0; c < 2; ++c)
+                for (int c = 0; c < NC; ++c)
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
 #pragma unroll
@@ -421,7 +495,7 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
             }
             float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
+            for (int c = 0; c < NC; ++c)
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     mx[0] = fmaxf(mx[0], fmaxf(__uint_as_float(sv[c][4 * k]), __uint_as_float(sv[c][4 * k + 1])));
@@ -454,7 +528,7 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                         l_part[k] *= f[k];
                     }
 #pragma unroll 1
-                    for (int cc = 0; cc < DC; cc += 64) {
+                    for (int cc = 0; cc + 64 <= DC; cc += 64) {
                         uint32_t o[32];
                         tmem_ld_16x256b_x8(tb + C::O_COL + cc, o);
                         tmem_wait_ld();
@@ -467,14 +541,27 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                         }
                         tmem_st_16x256b_x8(tb + C::O_COL + cc, o);
                     }
+                    if constexpr (DC % 64 != 0) {  // last 32 columns
+                        uint32_t o[16];
+                        tmem_ld_16x256b_x4(tb + C::O_COL + DC - 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            o[4 * k + 0] = __float_as_uint(__uint_as_float(o[4 * k + 0]) * f[0]);
+                            o[4 * k + 1] = __float_as_uint(__uint_as_float(o[4 * k + 1]) * f[0]);
+                            o[4 * k + 2] = __float_as_uint(__uint_as_float(o[4 * k + 2]) * f[1]);
+                            o[4 * k + 3] = __float_as_uint(__uint_as_float(o[4 * k + 3]) * f[1]);
+                        }
+                        tmem_st_16x256b_x4(tb + C::O_COL + DC - 32, o);
+                    }
                 }
             }
             // P = exp2(s * sl - m * sl), packed bf16 pairs for the 16x128b store:
             // rep kk (4 columns) <- pair (8k + 2 quad, +1) of column half c, kk = 8c + k
             const float nm0 = -m_used[0] * sl, nm1 = -m_used[1] * sl;
-            uint32_t pa[32];
+            uint32_t pa[2 * 8 * NC];
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
+            for (int c = 0; c < NC; ++c)
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const int kk = 8 * c + k;
@@ -492,7 +579,11 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                 if (!ok) break;
                 tc_fence_after();
             }
-            tmem_st_16x128b_x16(tb + C::P_COL, pa);
+            if constexpr (NC == 2) {
+                tmem_st_16x128b_x16(tb + C::P_COL, pa);
+            } else {
+                tmem_st_16x128b_x8(tb + C::P_COL, pa);
+            }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -510,30 +601,42 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                 lt[k] += __shfl_xor_sync(0xffffffffu, lt[k], 2);
                 inv[k] = 1.0f / lt[k];
             }
-            // O_lat = O / l as hi + lo bf16 parts, K-major SW128 operands in stages
-            // (nt+1) % NS and (nt+2) % NS (both drained: every PV has completed)
-            uint8_t* ol = stage((nt + 1) % NS);
+            // O_lat = O / l, K-major SW128: hi + lo bf16 parts in stages (nt+1) % NS and
+            // (nt+2) % NS, or (QS) one bf16 part in the Q region; all are idle: every S and
+            // PV MMA has completed
+            uint8_t* ol = C::QS ? qreg : stage((nt + 1) % NS);
             uint8_t* ol2 = stage((nt + 2) % NS);
             const int r_top = w4 * 32 + half * 16 + (lane >> 2);
             const int r_bot = r_top + 8;
 #pragma unroll 1
-            for (int cc = 0; cc < DC / 64; ++cc) {
+            for (int c32 = 0; c32 < DC / 32; c32 += 2) {  // 64 columns, or the last 32
                 uint32_t o[32];
-                tmem_ld_16x256b_x8(tb + C::O_COL + cc * 64, o);
+                const bool full = c32 + 2 <= DC / 32;
+                if (full) {
+                    tmem_ld_16x256b_x8(tb + C::O_COL + c32 * 32, o);
+                } else {
+                    tmem_ld_16x256b_x4(tb + C::O_COL + c32 * 32, *reinterpret_cast<uint32_t(*)[16]>(o));
+                }
                 tmem_wait_ld();
+                const int cc = c32 / 2;
                 const int off_top = cc * C::OLAT_ATOM + r_top * 128 + 4 * quad;
                 const int off_bot = cc * C::OLAT_ATOM + r_bot * 128 + 4 * quad;
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
+                    if (!full && k >= 4) break;
                     uint32_t hi, lo;
                     split_bf16(__uint_as_float(o[4 * k]) * inv[0], __uint_as_float(o[4 * k + 1]) * inv[0], hi, lo);
                     const int ot = off_top + ((k ^ (r_top & 7)) << 4);
-                    *reinterpret_cast<uint32_t*>(ol + ot) = hi;
-                    *reinterpret_cast<uint32_t*>(ol2 + ot) = lo;
+                    *reinterpret_cast<uint32_t*>(ol + ot) = C::QS ? pack_bf16(__uint_as_float(o[4 * k]) * inv[0],
+                                                                              __uint_as_float(o[4 * k + 1]) * inv[0])
+                                                                  : hi;
+                    if constexpr (!C::QS) *reinterpret_cast<uint32_t*>(ol2 + ot) = lo;
                     split_bf16(__uint_as_float(o[4 * k + 2]) * inv[1], __uint_as_float(o[4 * k + 3]) * inv[1], hi, lo);
                     const int ob = off_bot + ((k ^ (r_bot & 7)) << 4);
-                    *reinterpret_cast<uint32_t*>(ol + ob) = hi;
-                    *reinterpret_cast<uint32_t*>(ol2 + ob) = lo;
+                    *reinterpret_cast<uint32_t*>(ol + ob) = C::QS ? pack_bf16(__uint_as_float(o[4 * k + 2]) * inv[1],
+                                                                              __uint_as_float(o[4 * k + 3]) * inv[1])
+                                                                  : hi;
+                    if constexpr (!C::QS) *reinterpret_cast<uint32_t*>(ol2 + ob) = lo;
                 }
             }
             fence_proxy_async_smem();

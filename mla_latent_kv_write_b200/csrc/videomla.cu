@@ -392,6 +392,8 @@ int videomla_attention(const videomla_dims* dims, const void* q_nope, const void
     VMLA_AT(192, 32, 96, 128)
     VMLA_AT(192, 16, 112, 128)
     VMLA_AT(192, 64, 64, 128)
+    VMLA_AT(96, 32, 96, 128)
+    VMLA_AT(384, 32, 96, 128)
 #undef VMLA_AT
     return VIDEOMLA_EUNSUPPORTED;
 }

@@ -78,10 +78,11 @@ def test_attention_wan_wrapped_window_sampled_rows():
     _attention_case(dims, B=1, slots=21, oldest=13, n_valid=21, Nq=1560, seed=1002, rows=rows)
 
 
-@pytest.mark.parametrize("d_c,d_rope", [(192, 16), (192, 64)])
+@pytest.mark.parametrize("d_c,d_rope", [(96, 32), (192, 16), (192, 64), (384, 32)])
 def test_attention_sweep_points(d_c, d_rope):
     dims = dataclasses.replace(I.sweep_dims(d_c, d_rope), grid_h=6, grid_w=8)
-    _attention_case(dims, B=2, slots=5, oldest=3, n_valid=4, Nq=150, seed=4000 + d_rope)
+    seed = 4000 + d_rope + (0 if d_c == 192 else d_c)
+    _attention_case(dims, B=2, slots=5, oldest=3, n_valid=4, Nq=150, seed=seed)
 
 
 def test_attention_peaky_scores():
