@@ -128,33 +128,47 @@ def token_grid_position(p: np.ndarray, grid_w: int) -> Tuple[np.ndarray, np.ndar
     return p // grid_w, p % grid_w
 
 
-def window_keys(slots: int, oldest: int, n_valid: int, grid_h: int, grid_w: int):
+def window_keys(slots: int, oldest: int, n_valid: int, grid_h: int, grid_w: int, n_sink: int = 0):
     """Valid cache rows of the window in logical order, with their positions.
 
     The ring holds ``slots`` frames of T_f = grid_h * grid_w tokens; logical frame
     j (0 = oldest valid) lives in slot (oldest + j) mod slots.  [VideoMLA] App.
     D.5 gives the keys local temporal coordinates inside the current window:
     reading t = j.  Returns (rows[N], pos[N, 3]) with N = n_valid * T_f.
+
+    With ``n_sink`` pinned sink frames ([VideoMLA] App. D.4: one sink latent frame
+    plus a FIFO of the last frames) the cache rows are those of the sink frames,
+    rows [0, n_sink T_f), followed by the ring, rows n_sink T_f + (slot T_f + p).
+    The re-indexing of App. D.5 is read as: sink frame s at t = s, ring frame j at
+    t = n_sink + j, so the sink sits at local t = 0 before the FIFO frames.
     """
-    if not (1 <= n_valid <= slots and 0 <= oldest < slots):
+    if not (1 <= n_valid <= slots and 0 <= oldest < slots and n_sink >= 0):
         raise ValueError("bad window")
     T_f = grid_h * grid_w
     j = np.repeat(np.arange(n_valid), T_f)
     p = np.tile(np.arange(T_f), n_valid)
     slot = (oldest + j) % slots
-    rows = slot * T_f + p
+    rows = n_sink * T_f + slot * T_f + p
+    t = n_sink + j
+    if n_sink:
+        s_frame = np.repeat(np.arange(n_sink), T_f)
+        s_tok = np.tile(np.arange(T_f), n_sink)
+        rows = np.concatenate([s_frame * T_f + s_tok, rows])
+        t = np.concatenate([s_frame, t])
+        p = np.concatenate([s_tok, p])
     h, w = token_grid_position(p, grid_w)
-    return rows, np.stack([j, h, w], axis=-1)
+    return rows, np.stack([t, h, w], axis=-1)
 
 
-def window_queries(n_valid: int, n_query: int, grid_h: int, grid_w: int) -> np.ndarray:
+def window_queries(n_valid: int, n_query: int, grid_h: int, grid_w: int, n_sink: int = 0) -> np.ndarray:
     """Positions of the query chunk: the newest ``n_query`` tokens of the window
     in logical order, in the same local frame as the keys ([VideoMLA] App. D.5:
-    the current chunk is rotated in the same local coordinate system)."""
+    the current chunk is rotated in the same local coordinate system).  Sink
+    frames come first in that frame (see ``window_keys``)."""
     T_f = grid_h * grid_w
-    if not (1 <= n_query <= n_valid * T_f):
+    if not (1 <= n_query <= (n_sink + n_valid) * T_f):
         raise ValueError("bad query count")
-    L = n_valid * T_f - n_query + np.arange(n_query)
+    L = (n_sink + n_valid) * T_f - n_query + np.arange(n_query)
     h, w = token_grid_position(L % T_f, grid_w)
     return np.stack([L // T_f, h, w], axis=-1)
 
@@ -214,12 +228,12 @@ def _softmax_rows(s: np.ndarray):
 
 
 def _prepare(q_nope, q_rope, W_uk, W_uv, cache, slots, oldest, n_valid,
-             grid_h, grid_w, d_c, rope_base, pair_split, query_rows):
+             grid_h, grid_w, d_c, rope_base, pair_split, query_rows, n_sink):
     B, Nq, H, d_nope = q_nope.shape
     d_rope = q_rope.shape[-1]
     d_v = W_uv.shape[0] // H
-    rows, kpos = window_keys(slots, oldest, n_valid, grid_h, grid_w)
-    qpos = window_queries(n_valid, Nq, grid_h, grid_w)
+    rows, kpos = window_keys(slots, oldest, n_valid, grid_h, grid_w, n_sink)
+    qpos = window_queries(n_valid, Nq, grid_h, grid_w, n_sink)
     sel = np.arange(Nq) if query_rows is None else np.asarray(query_rows)
     omega, axis = rope_frequencies(d_rope, d_nope + d_rope, rope_base, pair_split)
     C = cache[:, rows, :d_c]                       # [B, N, d_c]
@@ -230,7 +244,7 @@ def _prepare(q_nope, q_rope, W_uk, W_uv, cache, slots, oldest, n_valid,
 
 def attention_explicit(q_nope, q_rope, W_uk, W_uv, cache, slots, oldest, n_valid,
                        grid_h, grid_w, d_c, rope_base=10000.0, pair_split=None,
-                       query_rows=None, return_probs=False):
+                       query_rows=None, return_probs=False, n_sink=0):
     """Training-time form ([VideoMLA] §3.3, Eq. 2, 6, 7; App. D.3-D.4).
 
     Per head h the keys and values are reconstructed from the cached latent:
@@ -245,10 +259,11 @@ def attention_explicit(q_nope, q_rope, W_uk, W_uv, cache, slots, oldest, n_valid
 
     Query rows are independent, so ``query_rows`` picks a subset of them; rows
     are processed in blocks only to bound memory, with identical arithmetic.
+    ``cache`` holds ``n_sink`` sink frames before the ring (see ``window_keys``).
     """
     B, H, d_nope, d_rope, d_v, sel, C, k_rope, q_rot = _prepare(
         q_nope, q_rope, W_uk, W_uv, cache, slots, oldest, n_valid, grid_h, grid_w,
-        d_c, rope_base, pair_split, query_rows)
+        d_c, rope_base, pair_split, query_rows, n_sink)
     scale = 1.0 / math.sqrt(d_nope + d_rope)
     out = np.empty((B, len(sel), H, d_v))
     lse = np.empty((B, len(sel), H))
@@ -271,7 +286,7 @@ def attention_explicit(q_nope, q_rope, W_uk, W_uv, cache, slots, oldest, n_valid
 
 def attention_absorbed(q_nope, q_rope, W_uk, W_uv, cache, slots, oldest, n_valid,
                        grid_h, grid_w, d_c, rope_base=10000.0, pair_split=None,
-                       query_rows=None):
+                       query_rows=None, n_sink=0):
     """Inference-time reparametrisation ([VideoMLA] App. E, Eq. 8-12).
 
     The key up-projection is absorbed into the query, q_abs = W_uk,h^T q^nope
@@ -283,7 +298,7 @@ def attention_absorbed(q_nope, q_rope, W_uk, W_uv, cache, slots, oldest, n_valid
     """
     B, H, d_nope, d_rope, d_v, sel, C, k_rope, q_rot = _prepare(
         q_nope, q_rope, W_uk, W_uv, cache, slots, oldest, n_valid, grid_h, grid_w,
-        d_c, rope_base, pair_split, query_rows)
+        d_c, rope_base, pair_split, query_rows, n_sink)
     scale = 1.0 / math.sqrt(d_nope + d_rope)
     out = np.empty((B, len(sel), H, d_v))
     lse = np.empty((B, len(sel), H))

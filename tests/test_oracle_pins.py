@@ -405,8 +405,8 @@ def test_pins_catch_dropped_rope_term(monkeypatch):
 
 def test_pins_catch_wrong_query_frame(monkeypatch):
     orig = O.window_queries
-    def shifted(n_valid, n_query, gh, gw):
-        q = orig(n_valid, n_query, gh, gw).copy(); q[:, 0] -= 1; return q
+    def shifted(n_valid, n_query, gh, gw, n_sink=0):
+        q = orig(n_valid, n_query, gh, gw, n_sink).copy(); q[:, 0] -= 1; return q
     assert _mutant_disagrees(monkeypatch, "window_queries", shifted)
 
 
@@ -418,8 +418,72 @@ def test_pins_catch_swapped_grid_axes(monkeypatch):
 
 def test_pins_catch_wrong_ring_order(monkeypatch):
     orig = O.window_keys
-    def reversed_t(slots, oldest, n_valid, gh, gw):
-        rows, pos = orig(slots, oldest, n_valid, gh, gw)
+    def reversed_t(slots, oldest, n_valid, gh, gw, n_sink=0):
+        rows, pos = orig(slots, oldest, n_valid, gh, gw, n_sink)
         pos = pos.copy(); pos[:, 0] = n_valid - 1 - pos[:, 0]
         return rows, pos
     assert _mutant_disagrees(monkeypatch, "window_keys", reversed_t)
+
+
+# ---------------------------------------------------------------------------
+# sink + FIFO window ([VideoMLA] App. D.4-D.5): one pinned sink frame before the
+# ring, re-indexed to local t = 0 with the FIFO frames at t = 1 .. n_valid
+# ---------------------------------------------------------------------------
+
+def _sink_problem(seed=11, Nq=8, oldest=2, n_valid=3):
+    prob = _tiny_problem(seed=seed, Nq=Nq, oldest=oldest, n_valid=n_valid)
+    T = TINY
+    T_f = T["grid_h"] * T["grid_w"]
+    rng = np.random.default_rng(seed + 1)
+    sink = rng.normal(size=(2, T_f, T["d_c"] + T["d_rope"]))
+    prob["cache"] = np.concatenate([sink, prob["cache"]], axis=1)   # sink rows first
+    return prob
+
+
+def test_sink_window_equals_brute_force_on_relaid_window():
+    """The sink window is the plain window whose logical frame 0 is the sink
+    frame and frames 1.. the FIFO frames oldest first: re-lay the cache that
+    way by hand and compare with the brute-force formulation."""
+    prob = _sink_problem()
+    T = TINY
+    T_f = T["grid_h"] * T["grid_w"]
+    slots, oldest, n_valid = prob["slots"], prob["oldest"], prob["n_valid"]
+    frames = [prob["cache"][:, 0:T_f]]                               # the sink
+    for j in range(n_valid):
+        slot = (oldest + j) % slots
+        frames.append(prob["cache"][:, T_f + slot * T_f:T_f + (slot + 1) * T_f])
+    relaid = dict(prob, cache=np.concatenate(frames, axis=1), slots=n_valid + 1, oldest=0, n_valid=n_valid + 1)
+    ref_out, ref_lse = _brute_force(**relaid)
+    out, lse = O.attention_absorbed(**prob, n_sink=1)
+    assert np.max(np.abs(out - ref_out)) < 1e-10
+    assert np.max(np.abs(lse - ref_lse)) < 1e-10
+    out_e, _ = O.attention_explicit(**prob, n_sink=1)
+    assert np.max(np.abs(out_e - ref_out)) < 1e-10
+
+
+def test_sink_window_positions():
+    T_f = 6
+    rows, pos = O.window_keys(slots=4, oldest=3, n_valid=2, grid_h=2, grid_w=3, n_sink=1)
+    assert rows.tolist() == list(range(6)) + [6 + 3 * 6 + p for p in range(6)] + [6 + 0 * 6 + p for p in range(6)]
+    assert pos[:T_f, 0].tolist() == [0] * T_f
+    assert pos[T_f:2 * T_f, 0].tolist() == [1] * T_f and pos[2 * T_f:, 0].tolist() == [2] * T_f
+    q = O.window_queries(n_valid=2, n_query=4, grid_h=2, grid_w=3, n_sink=1)
+    assert q[:, 0].tolist() == [2] * 4 and q[:, 1].tolist() == [0, 1, 1, 1]
+
+
+def test_sink_pin_catches_sink_after_fifo(monkeypatch):
+    """Placing the sink after the FIFO frames (t = n_valid) must be caught."""
+    prob = _sink_problem()
+    base_out, _ = O.attention_absorbed(**prob, n_sink=1)
+    orig = O.window_keys
+    def sink_last(slots, oldest, n_valid, gh, gw, n_sink=0):
+        rows, pos = orig(slots, oldest, n_valid, gh, gw, n_sink)
+        pos = pos.copy()
+        T_f = gh * gw
+        pos[:n_sink * T_f, 0] = n_valid + n_sink          # sink moved to the end
+        pos[n_sink * T_f:, 0] -= n_sink
+        return rows, pos
+    with monkeypatch.context() as m:
+        m.setattr(O, "window_keys", sink_last)
+        out, _ = O.attention_absorbed(**prob, n_sink=1)
+    assert np.max(np.abs(out - base_out)) > 1e-6
