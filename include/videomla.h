@@ -145,6 +145,42 @@ int videomla_attention(const videomla_dims* dims, const void* q_nope, const void
                        void* out, float* lse, void* workspace, size_t workspace_bytes,
                        void* stream);
 
+/* Largest number of pinned sink frames videomla_attention_sink accepts. */
+#define VIDEOMLA_MAX_SINK_FRAMES 8
+
+/*
+ * Bytes of the workspace that videomla_attention_sink needs: the rotated RoPE
+ * keys of the ring and of the sink frames, batch * (slots + n_sink) * T_f *
+ * d_rope fp16 values.  0 for invalid arguments.
+ */
+size_t videomla_attention_sink_workspace_size(const videomla_dims* dims, const videomla_window* window, int n_sink,
+                                              int batch);
+
+/*
+ * videomla_attention_sink -- videomla_attention over a sink-plus-window cache
+ * ("VideoMLA: Low-Rank Latent KV Cache for Minute-Scale Autoregressive Video
+ * Diffusion", App. D.4: one pinned sink latent frame plus a FIFO of the last
+ * frames; App. D.5: keys re-indexed to local temporal coordinates of that
+ * context).  The keys are the n_sink * T_f rows of ``sink_cache`` plus the
+ * n_valid * T_f valid rows of the ring ``cache``.  Local frame index: sink frame
+ * s is t = s, ring frame j (j frames after the oldest valid one) is
+ * t = n_sink + j; query i is logical token (n_sink + n_valid) * T_f - n_query + i.
+ *   sink_cache [batch, n_sink * T_f, d_c + d_rope] bf16, written like a ring of
+ *          n_sink slots by videomla_cache_write; may be NULL when n_sink == 0.
+ *   n_sink     0 .. VIDEOMLA_MAX_SINK_FRAMES (0 gives exactly videomla_attention).
+ *   workspace  at least videomla_attention_sink_workspace_size() bytes.
+ * Every other argument, the arithmetic and the launches are those of
+ * videomla_attention.
+ * Errors: EINVAL (as videomla_attention, plus n_sink out of range, sink_cache
+ * NULL or misaligned while n_sink > 0, n_query > (n_sink + n_valid) * T_f),
+ * EUNSUPPORTED, ECUDA.
+ */
+int videomla_attention_sink(const videomla_dims* dims, const void* q_nope, const void* q_rope,
+                            const void* W_uk, const void* W_uv, const void* cache,
+                            const videomla_window* window, const void* sink_cache, int n_sink,
+                            int batch, int n_query, void* out, float* lse, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
 /*
  * Bytes of the library's built-in scratch array used by
  * videomla_attention_static_workspace (16 MiB per device that loads the library).

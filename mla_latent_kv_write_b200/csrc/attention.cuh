@@ -39,7 +39,12 @@ namespace vmla {
 struct AttnParams {
     int Nq, H;
     int T_f, grid_w, slots, oldest;
-    int seg_start[2], seg_len[2];  // valid physical key rows: up to two contiguous runs
+    // valid key rows as up to three contiguous runs: runs 0 and 1 are physical
+    // rows of the ring cache (two when the ring wraps), run 2 the rows of the
+    // pinned sink frames (their own cache, rows [0, n_sink T_f))
+    int seg_start[3], seg_len[3];
+    int n_sink;                    // sink frames (local t = 0 .. n_sink-1; FIFO frames follow)
+    int ws_rows;                   // rotated-key workspace rows per batch element: (slots + n_sink) T_f
     int n_kt;                      // key tiles
     int q_first;                   // logical window index of query 0
     int n_t, n_h;                  // rope pairs of the t and h axes (w takes the rest)
@@ -52,11 +57,11 @@ struct AttnParams {
 };
 
 // TMA descriptors of one launch.  The key tensors get one map per valid run of
-// ring rows whose row extent ends at the end of the run, so a ragged last tile
-// reads zeros (never rows of slots outside the window).
+// rows whose row extent ends at the end of the run, so a ragged last tile reads
+// zeros (never rows of slots outside the window).
 struct AttnMaps {
-    CUtensorMap cc[2];  // cache latent part, per run: (d_c + d_rope, run rows, B), box (64, BK, 1), 128B swizzle
-    CUtensorMap kr[2];  // rotated rope keys (fp16), per run: (d_rope, run rows, B), box (d_rope, BK, 1)
+    CUtensorMap cc[3];  // cache latent part, per run: (d_c + d_rope, run rows, B), box (64, BK, 1), 128B swizzle
+    CUtensorMap kr[3];  // rotated rope keys (fp16), per run: (d_rope, run rows, B), box (d_rope, BK, 1)
     CUtensorMap qn;     // q_nope (d_nope, H, Nq, B), box (16, 1, BM, 1), 32B swizzle
     CUtensorMap wuk;    // W_uk (d_c, H * d_nope), box (64, d_nope), 128B swizzle
     CUtensorMap wuv;    // W_uv (d_c, H * d_v), box (64, d_v), 128B swizzle
@@ -124,8 +129,9 @@ struct AttnBarriers {
 template <int BK>
 __device__ __forceinline__ void key_tile(const AttnParams& p, int j, int& run, int& row, int& valid) {
     const int t0 = (p.seg_len[0] + BK - 1) / BK;
-    run = j < t0 ? 0 : 1;
-    row = (j < t0 ? j : j - t0) * BK;
+    const int t1 = t0 + (p.seg_len[1] + BK - 1) / BK;
+    run = j < t0 ? 0 : (j < t1 ? 1 : 2);
+    row = (j - (run == 0 ? 0 : run == 1 ? t0 : t1)) * BK;
     valid = min(BK, p.seg_len[run] - row);
 }
 
@@ -148,33 +154,50 @@ __device__ __forceinline__ float rope_theta(const AttnParams& p, int pr, int t, 
 
 // Forming the active window (App. D.5): rotate every valid cached k^R of the
 // window by its window-local (t, h, w) position, once per call, into the fp16
-// workspace [B, slots * T_f, DR] (same row indexing as the cache).  One thread
-// per (batch, valid row, 4 pairs).
+// workspace [B, (slots + n_sink) T_f, DR]: ring row R at row R, sink row r at
+// row slots T_f + r.  Local t: sink frame s -> s, ring frame j frames after the
+// oldest valid one -> n_sink + j (App. D.4-D.5).  One thread per (batch, valid
+// row, 4 pairs).
 template <int DC, int DR>
 __global__ void __launch_bounds__(256) rope_window_kernel(const __nv_bfloat16* __restrict__ cache,
+                                                          const __nv_bfloat16* __restrict__ sink,
                                                           __half* __restrict__ krot, const AttnParams p, int B) {
     constexpr int W = DC + DR, CH = DR / 8;
-    const int rows_valid = p.seg_len[0] + p.seg_len[1];
+    const int ring_valid = p.seg_len[0] + p.seg_len[1];
+    const int rows_valid = ring_valid + p.seg_len[2];
     const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (gid >= (long long)B * rows_valid * CH) return;
     const int ch = int(gid % CH);
     const long long t2 = gid / CH;
     const int vr = int(t2 % rows_valid);
     const int b = int(t2 / rows_valid);
-    const int R = vr < p.seg_len[0] ? p.seg_start[0] + vr : p.seg_start[1] + (vr - p.seg_len[0]);
-    const int slot = R / p.T_f;
-    const int pp = R - slot * p.T_f;
-    int t = slot - p.oldest;
-    if (t < 0) t += p.slots;
+    int t, pp;
+    const __nv_bfloat16* src;
+    size_t dst;
+    if (vr < ring_valid) {
+        const int R = vr < p.seg_len[0] ? p.seg_start[0] + vr : p.seg_start[1] + (vr - p.seg_len[0]);
+        const int slot = R / p.T_f;
+        pp = R - slot * p.T_f;
+        t = slot - p.oldest;
+        if (t < 0) t += p.slots;
+        t += p.n_sink;
+        src = cache + (size_t(b) * p.slots * p.T_f + R) * W;
+        dst = size_t(b) * p.ws_rows + R;
+    } else {
+        const int r = vr - ring_valid;
+        t = r / p.T_f;
+        pp = r - t * p.T_f;
+        src = sink + (size_t(b) * p.n_sink * p.T_f + r) * W;
+        dst = size_t(b) * p.ws_rows + size_t(p.slots) * p.T_f + r;
+    }
     const int hh = pp / p.grid_w, ww = pp - (pp / p.grid_w) * p.grid_w;
-    const size_t row = size_t(b) * p.slots * p.T_f + R;
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(cache + row * W + DC) + ch);
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + DC) + ch);
     uint4 o;
     o.x = rotate_pair(v.x, rope_theta(p, 4 * ch + 0, t, hh, ww));
     o.y = rotate_pair(v.y, rope_theta(p, 4 * ch + 1, t, hh, ww));
     o.z = rotate_pair(v.z, rope_theta(p, 4 * ch + 2, t, hh, ww));
     o.w = rotate_pair(v.w, rope_theta(p, 4 * ch + 3, t, hh, ww));
-    reinterpret_cast<uint4*>(krot + row * DR)[ch] = o;
+    reinterpret_cast<uint4*>(krot + dst * DR)[ch] = o;
 }
 
 template <class C>
@@ -224,7 +247,7 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            for (int r = 0; r < 2; ++r) {
+            for (int r = 0; r < 3; ++r) {
                 tma_prefetch_desc(&maps.cc[r]);
                 tma_prefetch_desc(&maps.kr[r]);
             }

@@ -222,7 +222,7 @@ int run_cache_write(const videomla_dims* d, const void* x, int B, int n_tok, con
 // attention
 // ----------------------------------------------------------------------------
 // Valid physical rows of the window: one run, or two when the ring wraps.
-void window_runs(const videomla_window* win, int T_f, int seg_start[2], int seg_len[2]) {
+void window_runs(const videomla_window* win, int T_f, int seg_start[3], int seg_len[3]) {
     seg_start[1] = seg_len[1] = 0;
     if (win->n_valid == win->slots) {
         seg_start[0] = 0;
@@ -240,8 +240,8 @@ void window_runs(const videomla_window* win, int T_f, int seg_start[2], int seg_
 
 template <int DC, int DR, int DN, int DV>
 int run_attention(const videomla_dims* d, const void* q_nope, const void* q_rope, const void* W_uk, const void* W_uv,
-                  const void* cache, const videomla_window* win, int B, int Nq, void* out, float* lse,
-                  void* workspace, cudaStream_t st) {
+                  const void* cache, const videomla_window* win, const void* sink, int n_sink, int B, int Nq,
+                  void* out, float* lse, void* workspace, cudaStream_t st) {
     using C = vmla::AttnCfg<DC, DR, DN, DV>;
     const int T_f = d->grid_h * d->grid_w;
     const int H = d->n_heads;
@@ -255,8 +255,13 @@ int run_attention(const videomla_dims* d, const void* q_nope, const void* q_rope
     p.slots = win->slots;
     p.oldest = win->oldest_slot;
     window_runs(win, T_f, p.seg_start, p.seg_len);
-    p.n_kt = (p.seg_len[0] + C::BK - 1) / C::BK + (p.seg_len[1] + C::BK - 1) / C::BK;
-    p.q_first = win->n_valid * T_f - Nq;
+    p.seg_start[2] = 0;
+    p.seg_len[2] = n_sink * T_f;
+    p.n_sink = n_sink;
+    p.ws_rows = (win->slots + n_sink) * T_f;
+    p.n_kt = 0;
+    for (int r = 0; r < 3; ++r) p.n_kt += (p.seg_len[r] + C::BK - 1) / C::BK;
+    p.q_first = (n_sink + win->n_valid) * T_f - Nq;
     p.n_t = d->pairs_t;
     p.n_h = d->pairs_h;
     // rope frequencies: an axis owning D_a dims of a full (d_nope + d_rope)-dim
@@ -281,18 +286,21 @@ int run_attention(const videomla_dims* d, const void* q_nope, const void* q_rope
     vmla::AttnMaps maps;
     const auto* cache_b = static_cast<const __nv_bfloat16*>(cache);
     const auto* krot = static_cast<const __half*>(workspace);
-    for (int r = 0; r < 2; ++r) {
-        const int run = p.seg_len[r] > 0 ? r : 0;  // an empty second run reuses the first (never read)
+    const auto* sink_b = static_cast<const __nv_bfloat16*>(sink);
+    for (int r = 0; r < 3; ++r) {
+        const int run = p.seg_len[r] > 0 ? r : 0;  // an empty run reuses the first (never read)
+        const bool is_sink = run == 2;
+        const __nv_bfloat16* base = is_sink ? sink_b : cache_b + size_t(p.seg_start[run]) * C::W;
+        const uint64_t batch_rows = is_sink ? uint64_t(n_sink) * T_f : uint64_t(rows);
         const uint64_t dc[3] = {uint64_t(C::W), uint64_t(p.seg_len[run]), uint64_t(B)};
-        const uint64_t sc[2] = {uint64_t(C::W) * 2, uint64_t(rows) * C::W * 2};
+        const uint64_t sc[2] = {uint64_t(C::W) * 2, batch_rows * C::W * 2};
         const uint32_t bc[3] = {64, uint32_t(C::BK), 1};
-        if (!make_map(&maps.cc[r], cache_b + size_t(p.seg_start[run]) * C::W, 3, dc, sc, bc, 128))
-            return VIDEOMLA_ECUDA;
+        if (!make_map(&maps.cc[r], base, 3, dc, sc, bc, 128)) return VIDEOMLA_ECUDA;
+        const size_t ws_row0 = is_sink ? size_t(rows) : size_t(p.seg_start[run]);
         const uint64_t dr[3] = {uint64_t(DR), uint64_t(p.seg_len[run]), uint64_t(B)};
-        const uint64_t sr[2] = {uint64_t(DR) * 2, uint64_t(rows) * DR * 2};
+        const uint64_t sr[2] = {uint64_t(DR) * 2, uint64_t(p.ws_rows) * DR * 2};
         const uint32_t br[3] = {uint32_t(DR), uint32_t(C::BK), 1};
-        if (!make_map(&maps.kr[r], krot + size_t(p.seg_start[run]) * DR, 3, dr, sr, br, DR * 2,
-                      CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+        if (!make_map(&maps.kr[r], krot + ws_row0 * DR, 3, dr, sr, br, DR * 2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
             return VIDEOMLA_ECUDA;
     }
     {
@@ -315,9 +323,9 @@ int run_attention(const videomla_dims* d, const void* q_nope, const void* q_rope
     }
     // 1) form the window: rotated rope keys into the workspace
     {
-        const long long work = (long long)B * (p.seg_len[0] + p.seg_len[1]) * (DR / 8);
+        const long long work = (long long)B * (p.seg_len[0] + p.seg_len[1] + p.seg_len[2]) * (DR / 8);
         const int blocks = int((work + 255) / 256);
-        vmla::rope_window_kernel<DC, DR><<<blocks, 256, 0, st>>>(cache_b, static_cast<__half*>(workspace), p, B);
+        vmla::rope_window_kernel<DC, DR><<<blocks, 256, 0, st>>>(cache_b, sink_b, static_cast<__half*>(workspace), p, B);
     }
     // 2) latent attention
     auto kern = vmla::attention_kernel<C>;
@@ -360,25 +368,33 @@ int videomla_cache_write(const videomla_dims* dims, const void* x, int batch, in
     return VIDEOMLA_EUNSUPPORTED;
 }
 
-size_t videomla_attention_workspace_size(const videomla_dims* dims, const videomla_window* window, int batch) {
-    if (!dims || !window || batch <= 0 || window->slots <= 0 || dims->grid_h <= 0 || dims->grid_w <= 0 ||
-        dims->d_rope <= 0)
+size_t videomla_attention_sink_workspace_size(const videomla_dims* dims, const videomla_window* window, int n_sink,
+                                              int batch) {
+    if (!dims || !window || batch <= 0 || window->slots <= 0 || n_sink < 0 || dims->grid_h <= 0 ||
+        dims->grid_w <= 0 || dims->d_rope <= 0)
         return 0;
-    return size_t(batch) * window->slots * size_t(dims->grid_h) * dims->grid_w * dims->d_rope * 2;
+    return size_t(batch) * (window->slots + n_sink) * size_t(dims->grid_h) * dims->grid_w * dims->d_rope * 2;
 }
 
-int videomla_attention(const videomla_dims* dims, const void* q_nope, const void* q_rope, const void* W_uk,
-                       const void* W_uv, const void* cache, const videomla_window* window, int batch, int n_query,
-                       void* out, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+size_t videomla_attention_workspace_size(const videomla_dims* dims, const videomla_window* window, int batch) {
+    return videomla_attention_sink_workspace_size(dims, window, 0, batch);
+}
+
+int videomla_attention_sink(const videomla_dims* dims, const void* q_nope, const void* q_rope, const void* W_uk,
+                            const void* W_uv, const void* cache, const videomla_window* window, const void* sink_cache,
+                            int n_sink, int batch, int n_query, void* out, float* lse, void* workspace,
+                            size_t workspace_bytes, void* stream) {
     if (!basic_dims_ok(dims) || !q_nope || !q_rope || !W_uk || !W_uv || !cache || !window || !out || !workspace)
         return VIDEOMLA_EINVAL;
     const videomla_window w = *window;
     if (w.slots <= 0 || w.oldest_slot < 0 || w.oldest_slot >= w.slots || w.n_valid < 1 || w.n_valid > w.slots)
         return VIDEOMLA_EINVAL;
+    if (n_sink < 0 || n_sink > VIDEOMLA_MAX_SINK_FRAMES || (n_sink > 0 && (!sink_cache || !aligned16(sink_cache))))
+        return VIDEOMLA_EINVAL;
     const long long T_f = (long long)dims->grid_h * dims->grid_w;
-    if (batch <= 0 || batch > 65535 || n_query <= 0 || n_query > w.n_valid * T_f) return VIDEOMLA_EINVAL;
-    if ((long long)w.slots * T_f > (1ll << 30) || dims->n_heads > 65535) return VIDEOMLA_EINVAL;
-    if (workspace_bytes < videomla_attention_workspace_size(dims, window, batch)) return VIDEOMLA_EINVAL;
+    if (batch <= 0 || batch > 65535 || n_query <= 0 || n_query > (n_sink + w.n_valid) * T_f) return VIDEOMLA_EINVAL;
+    if ((long long)(w.slots + n_sink) * T_f > (1ll << 30) || dims->n_heads > 65535) return VIDEOMLA_EINVAL;
+    if (workspace_bytes < videomla_attention_sink_workspace_size(dims, window, n_sink, batch)) return VIDEOMLA_EINVAL;
     if (!aligned16(q_nope) || !aligned16(q_rope) || !aligned16(W_uk) || !aligned16(W_uv) || !aligned16(cache) ||
         !aligned16(out) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(lse) & 3u))
         return VIDEOMLA_EINVAL;
@@ -387,8 +403,8 @@ int videomla_attention(const videomla_dims* dims, const void* q_nope, const void
     const int dc = dims->d_c, dr = dims->d_rope, dn = dims->d_nope, dv = dims->d_v;
 #define VMLA_AT(DC_, DR_, DN_, DV_)                        \
     if (dc == DC_ && dr == DR_ && dn == DN_ && dv == DV_) \
-        return run_attention<DC_, DR_, DN_, DV_>(dims, q_nope, q_rope, W_uk, W_uv, cache, &w, batch, n_query, out, lse, \
-                                                 workspace, st);
+        return run_attention<DC_, DR_, DN_, DV_>(dims, q_nope, q_rope, W_uk, W_uv, cache, &w, sink_cache, n_sink, \
+                                                 batch, n_query, out, lse, workspace, st);
     VMLA_AT(192, 32, 96, 128)
     VMLA_AT(192, 16, 112, 128)
     VMLA_AT(192, 64, 64, 128)
@@ -396,6 +412,13 @@ int videomla_attention(const videomla_dims* dims, const void* q_nope, const void
     VMLA_AT(384, 32, 96, 128)
 #undef VMLA_AT
     return VIDEOMLA_EUNSUPPORTED;
+}
+
+int videomla_attention(const videomla_dims* dims, const void* q_nope, const void* q_rope, const void* W_uk,
+                       const void* W_uv, const void* cache, const videomla_window* window, int batch, int n_query,
+                       void* out, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+    return videomla_attention_sink(dims, q_nope, q_rope, W_uk, W_uv, cache, window, nullptr, 0, batch, n_query, out,
+                                   lse, workspace, workspace_bytes, stream);
 }
 
 }  // extern "C"

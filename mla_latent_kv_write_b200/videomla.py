@@ -29,6 +29,8 @@ EXPORTED = (
     "videomla_attention",
     "videomla_attention_workspace_size",
     "videomla_attention_static_workspace",
+    "videomla_attention_sink",
+    "videomla_attention_sink_workspace_size",
     "videomla_strerror",
     "videomla_device_status",
     "videomla_set_wait_timeout_ns",
@@ -75,6 +77,11 @@ def load_library() -> ctypes.CDLL:
         lib.videomla_attention.restype = ci
         lib.videomla_attention_workspace_size.argtypes = [ctypes.POINTER(CDims), ctypes.POINTER(CWindow), ci]
         lib.videomla_attention_workspace_size.restype = ctypes.c_size_t
+        lib.videomla_attention_sink.argtypes = [ctypes.POINTER(CDims), vp, vp, vp, vp, vp, ctypes.POINTER(CWindow),
+                                                vp, ci, ci, ci, vp, vp, vp, ctypes.c_size_t, vp]
+        lib.videomla_attention_sink.restype = ci
+        lib.videomla_attention_sink_workspace_size.argtypes = [ctypes.POINTER(CDims), ctypes.POINTER(CWindow), ci, ci]
+        lib.videomla_attention_sink_workspace_size.restype = ctypes.c_size_t
         lib.videomla_strerror.argtypes = [ci]
         lib.videomla_strerror.restype = ctypes.c_char_p
         lib.videomla_device_status.argtypes = [ci]
@@ -150,19 +157,23 @@ def cache_write(x: torch.Tensor, W_dkv: torch.Tensor, W_kr: torch.Tensor, gamma:
     return cache
 
 
-def workspace_size(dims: Dims, slots: int, oldest: int, n_valid: int, batch: int) -> int:
+def workspace_size(dims: Dims, slots: int, oldest: int, n_valid: int, batch: int, n_sink: int = 0) -> int:
     """Bytes of the attention workspace (the window's rotated RoPE keys)."""
     cd, win = c_dims(dims), CWindow(slots, oldest, n_valid)
-    return int(load_library().videomla_attention_workspace_size(ctypes.byref(cd), ctypes.byref(win), batch))
+    return int(load_library().videomla_attention_sink_workspace_size(ctypes.byref(cd), ctypes.byref(win), n_sink,
+                                                                     batch))
 
 
 def attention(q_nope: torch.Tensor, q_rope: torch.Tensor, W_uk: torch.Tensor, W_uv: torch.Tensor,
               cache: torch.Tensor, dims: Dims, slots: int, oldest: int, n_valid: int,
               out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-              want_lse: bool = False, workspace: Optional[torch.Tensor] = None, stream=None):
+              want_lse: bool = False, workspace: Optional[torch.Tensor] = None, stream=None,
+              sink: Optional[torch.Tensor] = None):
     """Latent attention of the queries over the window; returns ``out``
     [B, Nq, H, d_v] (and ``lse`` [B, Nq, H] if requested or given).
 
+    ``sink`` [B, n_sink T_f, d_c + d_rope] holds pinned sink frames that join
+    the window before the ring frames (``videomla_attention_sink``).
     ``workspace`` is a device byte buffer of at least ``workspace_size(...)``
     bytes; if omitted, one is taken from torch's stream-ordered caching
     allocator for this call."""
@@ -181,18 +192,31 @@ def attention(q_nope: torch.Tensor, q_rope: torch.Tensor, W_uk: torch.Tensor, W_
         lse = torch.empty(B, Nq, H, dtype=torch.float32, device=dev)
     if lse is not None:
         _check(lse, "lse", torch.float32, (B, Nq, H), dev)
+    T_f = dims.tokens_per_frame
+    n_sink = 0
+    if sink is not None:
+        if sink.dim() != 3 or sink.shape[1] % T_f != 0:
+            raise ValueError("sink must be [B, n_sink * T_f, d_c + d_rope]")
+        n_sink = sink.shape[1] // T_f
+        _check(sink, "sink", torch.bfloat16, (B, n_sink * T_f, dims.cache_width), dev)
     cd = c_dims(dims)
     win = CWindow(slots, oldest, n_valid)
-    need = int(lib.videomla_attention_workspace_size(ctypes.byref(cd), ctypes.byref(win), B))
+    need = int(lib.videomla_attention_sink_workspace_size(ctypes.byref(cd), ctypes.byref(win), n_sink, B))
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     elif workspace.device != dev or workspace.numel() * workspace.element_size() < need:
         raise ValueError(f"workspace must be a {need}-byte buffer on {dev}")
-    rc = lib.videomla_attention(ctypes.byref(cd), _ptr(q_nope), _ptr(q_rope), _ptr(W_uk), _ptr(W_uv),
-                                _ptr(cache), ctypes.byref(win), B, Nq, _ptr(out), _ptr(lse), _ptr(workspace),
-                                workspace.numel() * workspace.element_size(), _stream(stream))
+    if sink is None:
+        rc = lib.videomla_attention(ctypes.byref(cd), _ptr(q_nope), _ptr(q_rope), _ptr(W_uk), _ptr(W_uv),
+                                    _ptr(cache), ctypes.byref(win), B, Nq, _ptr(out), _ptr(lse), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream))
+    else:
+        rc = lib.videomla_attention_sink(ctypes.byref(cd), _ptr(q_nope), _ptr(q_rope), _ptr(W_uk), _ptr(W_uv),
+                                         _ptr(cache), ctypes.byref(win), _ptr(sink), n_sink, B, Nq, _ptr(out),
+                                         _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                         _stream(stream))
     if rc != OK:
-        raise VideoMLAError(rc, "videomla_attention")
+        raise VideoMLAError(rc, "videomla_attention_sink" if sink is not None else "videomla_attention")
     return (out, lse) if lse is not None else out
 
 

@@ -46,10 +46,17 @@ def to_bf16(a: np.ndarray) -> torch.Tensor:
 
 
 def oracle_attention(dims: I.Dims, q: dict, w: dict, cache_bf16: torch.Tensor, slots: int, oldest: int,
-                     n_valid: int, rows=None):
+                     n_valid: int, rows=None, sink_bf16: torch.Tensor = None):
+    """The oracle's absorbed form; pinned sink frames (``sink_bf16`` [B, n_sink T_f, W])
+    go before the ring rows, the layout the oracle's window functions read."""
+    cache = f64(cache_bf16)
+    n_sink = 0
+    if sink_bf16 is not None:
+        n_sink = sink_bf16.shape[1] // dims.tokens_per_frame
+        cache = np.concatenate([f64(sink_bf16), cache], axis=1)
     return O.attention_absorbed(f64(q["q_nope"]), f64(q["q_rope"]), f64(w["W_uk"]), f64(w["W_uv"]),
-                                f64(cache_bf16), slots, oldest, n_valid, dims.grid_h, dims.grid_w, dims.d_c,
-                                dims.rope_base, dims.pairs, query_rows=rows)
+                                cache, slots, oldest, n_valid, dims.grid_h, dims.grid_w, dims.d_c,
+                                dims.rope_base, dims.pairs, query_rows=rows, n_sink=n_sink)
 
 
 def check_attention(got: np.ndarray, ref: np.ndarray, what: str = ""):

@@ -134,3 +134,23 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(V, "_LIB", None)
     with pytest.raises(V.VideoMLAError):
         V.load_library()
+
+
+def test_attention_sink_rejects_bad_arguments(lib):
+    d = _dims()
+    win = V.CWindow(6, 0, 6)
+    P = ctypes.c_void_p(0x10000)
+    T_f = d.grid_h * d.grid_w
+    ws = lib.videomla_attention_sink_workspace_size(ctypes.byref(d), ctypes.byref(win), 1, 1)
+    assert ws == (6 + 1) * T_f * d.d_rope * 2
+    assert lib.videomla_attention_workspace_size(ctypes.byref(d), ctypes.byref(win), 1) == 6 * T_f * d.d_rope * 2
+
+    def call(sink=P, n_sink=1, nq=T_f, ws_bytes=ws):
+        return lib.videomla_attention_sink(ctypes.byref(d), P, P, P, P, P, ctypes.byref(win), sink, n_sink, 1, nq, P,
+                                           None, P, ws_bytes, None)
+    assert call(n_sink=-1) == V.EINVAL
+    assert call(n_sink=9) == V.EINVAL                              # above VIDEOMLA_MAX_SINK_FRAMES
+    assert call(sink=None) == V.EINVAL                             # sink cache missing
+    assert call(sink=ctypes.c_void_p(0x10008)) == V.EINVAL         # misaligned sink cache
+    assert call(nq=7 * T_f + 1) == V.EINVAL                        # more queries than sink + window tokens
+    assert call(ws_bytes=ws - 1) == V.EINVAL                       # workspace without the sink rows

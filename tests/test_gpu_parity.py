@@ -24,20 +24,22 @@ def _dev(d):
     return {k: v.to(DEV) for k, v in d.items()}
 
 
-def _attention_case(dims, B, slots, oldest, n_valid, Nq, seed, rows=None, rope_scale=1.0):
+def _attention_case(dims, B, slots, oldest, n_valid, Nq, seed, rows=None, rope_scale=1.0, n_sink=0):
     w = I.layer_weights(dims, seed)
     q = I.queries(dims, B, Nq, seed + 1)
     cache = I.latent_cache(dims, B, slots, seed + 2, rope_scale=rope_scale)
+    sink = I.latent_cache(dims, B, n_sink, seed + 3, rope_scale=rope_scale) if n_sink else None
     wd, qd = _dev(w), _dev(q)
     out, lse = V.attention(qd["q_nope"], qd["q_rope"], wd["W_uk"], wd["W_uv"], cache.to(DEV), dims,
-                           slots, oldest, n_valid, want_lse=True)
+                           slots, oldest, n_valid, want_lse=True, sink=None if sink is None else sink.to(DEV))
     torch.cuda.synchronize()
     assert V.device_status(reset=True) == V.OK
-    ref_out, ref_lse = oracle_attention(dims, q, w, cache, slots, oldest, n_valid, rows)
+    ref_out, ref_lse = oracle_attention(dims, q, w, cache, slots, oldest, n_valid, rows, sink_bf16=sink)
     got_out, got_lse = f64(out.cpu()), f64(lse.cpu())
     if rows is not None:
         got_out, got_lse = got_out[:, rows], got_lse[:, rows]
-    what = f"attention {dims.d_c}/{dims.d_rope} B={B} slots={slots} oldest={oldest} n_valid={n_valid} Nq={Nq}"
+    what = (f"attention {dims.d_c}/{dims.d_rope} B={B} slots={slots} oldest={oldest} n_valid={n_valid} Nq={Nq}"
+            f"{f' sink={n_sink}' if n_sink else ''}")
     err = got_out - ref_out
     print(f"\n{what}: rms rel {np.linalg.norm(err) / np.linalg.norm(ref_out):.2e} "
           f"max abs {np.max(np.abs(err)):.2e} lse {np.max(np.abs(got_lse - ref_lse)):.2e}")
@@ -83,6 +85,28 @@ def test_attention_sweep_points(d_c, d_rope):
     dims = dataclasses.replace(I.sweep_dims(d_c, d_rope), grid_h=6, grid_w=8)
     seed = 4000 + d_rope + (0 if d_c == 192 else d_c)
     _attention_case(dims, B=2, slots=5, oldest=3, n_valid=4, Nq=150, seed=seed)
+
+
+@pytest.mark.parametrize("slots,oldest,n_valid,Nq,B", [
+    (6, 4, 6, 144, 2),    # sink + full wrapping FIFO: three runs of key rows, ragged tiles
+    (6, 0, 2, 96, 1),     # sink + FIFO not yet full
+    (4, 3, 3, 192, 1),    # queries reach back into the sink frame
+])
+def test_attention_sink_window(slots, oldest, n_valid, Nq, B):
+    _attention_case(I.TINY, B=B, slots=slots, oldest=oldest, n_valid=n_valid, Nq=Nq, seed=21 + slots + oldest,
+                    n_sink=1)
+
+
+def test_attention_sink_window_q_in_shared_memory():
+    dims = dataclasses.replace(I.sweep_dims(384, 32), grid_h=6, grid_w=8)
+    _attention_case(dims, B=2, slots=4, oldest=1, n_valid=4, Nq=96, seed=4500, n_sink=1)
+
+
+def test_attention_wan_sink_plus_six_frames_sampled_rows():
+    """The pages' inference cache: one sink latent frame plus a FIFO of six
+    (10,920 keys), the 3-frame chunk as queries, a wrapped FIFO."""
+    rows = sample_rows(4680, 64, seed=7)
+    _attention_case(I.WAN, B=1, slots=6, oldest=2, n_valid=6, Nq=4680, seed=1003, rows=rows, n_sink=1)
 
 
 def test_attention_peaky_scores():
