@@ -347,6 +347,10 @@ def run_gpu(args):
     cw_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     clocks = clk.summary()
 
+    s0 = sets[0]
+    h2d_bytes = sum(s0[n].numel() * s0[n].element_size() for n in ("x", "q_nope", "q_rope"))
+    d2h_bytes = s0["out"].numel() * s0["out"].element_size()
+
     # ---- end to end through host buffers
     for i in range(max(1, args.warmup)):
         step_e2e(sets[i % N_SETS])
@@ -363,10 +367,11 @@ def run_gpu(args):
 
     # ---- cache_write on a 30-layer stack (494 MB > L2), for its HBM roofline
     cw_stack = cache_write_stack(dev)
+    del sets
+    side = side_workloads(dev, measured_peaks()[0]["bf16_tflops"]) if world == 1 and not args.no_side else {}
 
-    s0 = sets[0]
-    h2d = sum(s0[n].numel() * s0[n].element_size() for n in ("x", "q_nope", "q_rope"))
-    d2h = s0["out"].numel() * s0["out"].element_size()
+    h2d = h2d_bytes
+    d2h = d2h_bytes
 
     if rank == 0:
         peaks, peak_src = measured_peaks()
@@ -399,6 +404,7 @@ def run_gpu(args):
             "explicit_mha_equivalent_tflops": flops_explicit_equivalent(d, wl.batch, wl.n_query, Nk)
             / (attn_ms * 1e-3) / 1e12,
             "cache_write_stack": cw_stack,
+            **side,
             "e2e": {"value": job_throughput(world, fl_step, e2e_ms, args.steps) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                     "ms_per_step": e2e_ms / args.steps},
@@ -413,6 +419,64 @@ def run_gpu(args):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def _time_attention_calls(calls, reps: int):
+    """Mean ms of one call of each of ``calls`` (closures launching one attention
+    call), cycled ``reps`` times after a warm-up round; CUDA events on the
+    current stream, which is the stream the calls launch on."""
+    for c in calls:
+        c()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        for c in calls:
+            c()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / (reps * len(calls))
+
+
+def side_workloads(dev, peak: float):
+    """Attention on the pages' inference cache (one sink frame + a FIFO of six,
+    App. D.4) and on every (d_c, d_rope) point of the rank / RoPE sweep (3 query
+    frames vs a 21-frame window); each with 4 rotating input sets."""
+    from mla_latent_kv_write_b200 import videomla as V
+    wl = WORKLOAD
+    res = {}
+
+    def make(d, slots, n_sink, k):
+        T_f = d.tokens_per_frame
+        seed = I.seed_for(5, k, slots)
+        w = {n: t.to(dev) for n, t in I.layer_weights(d, seed).items()}
+        q = {n: t.to(dev) for n, t in I.queries(d, 1, wl.n_query, seed + 1).items()}
+        cache = I.latent_cache(d, 1, slots, seed + 2).to(dev)
+        sink = I.latent_cache(d, 1, n_sink, seed + 3).to(dev) if n_sink else None
+        ws = torch.empty(V.workspace_size(d, slots, 0, slots, 1, n_sink), dtype=torch.uint8, device=dev)
+        out = torch.empty(1, wl.n_query, d.n_heads, d.d_v, dtype=torch.bfloat16, device=dev)
+        return lambda: V.attention(q["q_nope"], q["q_rope"], w["W_uk"], w["W_uv"], cache, d, slots, 0, slots,
+                                   out=out, workspace=ws, sink=sink)
+
+    d = wl.dims
+    calls = [make(d, 6, 1, k) for k in range(N_SETS)]
+    ms = _time_attention_calls(calls, 10)
+    Nk = 7 * d.tokens_per_frame
+    tf = flops_attention(d, 1, wl.n_query, Nk) / (ms * 1e-3) / 1e12
+    res["sink_window"] = {"workload": "Wan layer, 1 sink frame + FIFO of 6 frames (10920 keys), 4680 queries",
+                          "ms": ms, "tflops": tf, "frac": tf / peak}
+    del calls
+    sweep = []
+    for d_c, d_rope in I.SWEEP_POINTS:
+        ds = I.sweep_dims(d_c, d_rope)
+        calls = [make(ds, wl.slots, 0, k) for k in range(2)]
+        ms = _time_attention_calls(calls, 5)
+        tf = flops_attention(ds, 1, wl.n_query, wl.slots * ds.tokens_per_frame) / (ms * 1e-3) / 1e12
+        sweep.append({"d_c": d_c, "d_rope": d_rope, "ms": ms, "tflops": tf, "frac": tf / peak})
+        del calls
+    res["sweep_attention"] = sweep
+    torch.cuda.empty_cache()
+    return res
 
 
 def cache_write_stack(dev, layers: int = 30, reps: int = 3):
@@ -471,6 +535,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-side", action="store_true", help="skip the sink-window and sweep side measurements")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
