@@ -298,13 +298,51 @@ def step(s, ev=None):
         ev[2].record()
 
 
-def step_e2e(s):
-    """Same step through the public API with host buffers: H2D of the step's
-    inputs (x, q_nope, q_rope) from pinned memory, the two kernels, D2H of out."""
-    for name in ("x", "q_nope", "q_rope"):
-        s[name].copy_(s[name + "_host"], non_blocking=True)
-    step(s)
-    s["out_host"].copy_(s["out"], non_blocking=True)
+def run_e2e(sets, n_steps: int):
+    """``n_steps`` steps through the public API with host buffers, pipelined the
+    way a server would run them: step i's inputs (x, q_nope, q_rope) go up from
+    pinned memory on a copy stream while step i-1 computes, step i's output
+    comes back on a second copy stream while step i+1 computes.  Events keep
+    every buffer set's reuse ordered (4 rotating sets).  Returns the elapsed ms
+    from the first upload to the last download, timed with events recorded on
+    the compute stream after it joined both copy streams."""
+    comp = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    n = len(sets)
+    ev = lambda: torch.cuda.Event()
+    ev_in, ev_done, ev_out = {}, {}, {}
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    up.wait_stream(comp)
+    down.wait_stream(comp)
+    start.record(up)
+
+    def upload(i):
+        s = sets[i % n]
+        if i - n in ev_done:                 # the set's previous step has finished reading it
+            up.wait_event(ev_done[i - n])
+        with torch.cuda.stream(up):
+            for name in ("x", "q_nope", "q_rope"):
+                s[name].copy_(s[name + "_host"], non_blocking=True)
+        ev_in[i] = ev(); ev_in[i].record(up)
+
+    upload(0)
+    for i in range(n_steps):
+        if i + 1 < n_steps:
+            upload(i + 1)
+        comp.wait_event(ev_in[i])
+        if i - n in ev_out:                  # the set's previous output has been downloaded
+            comp.wait_event(ev_out[i - n])
+        step(sets[i % n])
+        ev_done[i] = ev(); ev_done[i].record(comp)
+        down.wait_event(ev_done[i])
+        with torch.cuda.stream(down):
+            sets[i % n]["out_host"].copy_(sets[i % n]["out"], non_blocking=True)
+        ev_out[i] = ev(); ev_out[i].record(down)
+    comp.wait_stream(up)
+    comp.wait_stream(down)
+    stop.record(comp)
+    torch.cuda.synchronize()
+    return start.elapsed_time(stop)
 
 
 def run_gpu(args):
@@ -351,17 +389,12 @@ def run_gpu(args):
     h2d_bytes = sum(s0[n].numel() * s0[n].element_size() for n in ("x", "q_nope", "q_rope"))
     d2h_bytes = s0["out"].numel() * s0["out"].element_size()
 
-    # ---- end to end through host buffers
-    for i in range(max(1, args.warmup)):
-        step_e2e(sets[i % N_SETS])
+    # ---- end to end through host buffers (uploads / downloads pipelined with compute)
+    run_e2e(sets, max(1, args.warmup))
     barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(args.steps):
-        step_e2e(sets[i % N_SETS])
-    e1.record()
+    e2e_local = run_e2e(sets, args.steps)
     barrier(world)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_ms = max_over_ranks(e2e_local, world)
     if V.device_status(reset=True) != V.OK:
         raise RuntimeError("a kernel reported a timed-out device wait")
 
@@ -407,7 +440,8 @@ def run_gpu(args):
             **side,
             "e2e": {"value": job_throughput(world, fl_step, e2e_ms, args.steps) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-                    "ms_per_step": e2e_ms / args.steps},
+                    "ms_per_step": e2e_ms / args.steps,
+                    "pipelining": "step i+1 upload and step i-1 download overlap step i's kernels"},
             "clocks": clocks,
             "gpu_launches": 3 * args.steps,  # cache_write, window pre-pass, attention
         }
@@ -476,7 +510,42 @@ def side_workloads(dev, peak: float):
         del calls
     res["sweep_attention"] = sweep
     torch.cuda.empty_cache()
+    res["dense_mha_library"] = dense_mha_library(dev, d, wl.n_query, wl.slots * d.tokens_per_frame)
     return res
+
+
+def dense_mha_library(dev, d, Nq: int, Nk: int):
+    """Same-shape dense multi-head attention through torch's scaled-dot-product
+    attention (a library kernel, not this repository's): per-head K and V of
+    d_nope + d_rope = 128 channels for every key, the 2 n_h d_h = 3072-scalar
+    cache of the pages' dense baseline ([VideoMLA] App. C.1).  For the same-box
+    time and cache-bytes ratios only; its flops are 4 d_h per (q, k, h)."""
+    import torch.nn.functional as F
+    dh = d.d_nope + d.d_rope
+    g = torch.Generator(device="cpu").manual_seed(77)
+    sets = []
+    for _ in range(2):   # 2 x 2 x 201 MB of K / V: larger than L2
+        q = torch.randn(1, d.n_heads, Nq, dh, generator=g).to(torch.bfloat16).to(dev)
+        k = torch.randn(1, d.n_heads, Nk, dh, generator=g).to(torch.bfloat16).to(dev)
+        v = torch.randn(1, d.n_heads, Nk, dh, generator=g).to(torch.bfloat16).to(dev)
+        sets.append((q, k, v))
+    backend = "default"
+    try:
+        from torch.nn.attention import SDPBackend, sdpa_kernel
+        ctx = sdpa_kernel([SDPBackend.CUDNN_ATTENTION, SDPBackend.FLASH_ATTENTION, SDPBackend.EFFICIENT_ATTENTION])
+        backend = "cudnn / flash / efficient (first available)"
+    except Exception:  # older torch: its own choice
+        import contextlib
+        ctx = contextlib.nullcontext()
+    with ctx:
+        calls = [lambda q=q, k=k, v=v: F.scaled_dot_product_attention(q, k, v) for q, k, v in sets]
+        ms = _time_attention_calls(calls, 5)
+    fl = 4.0 * dh * Nq * Nk * d.n_heads
+    del sets
+    torch.cuda.empty_cache()
+    return {"what": "torch scaled_dot_product_attention on per-head K / V (library kernel)", "backend": backend,
+            "ms": ms, "tflops": fl / (ms * 1e-3) / 1e12, "cache_bytes_per_token_layer": 2 * 2 * d.n_heads * dh,
+            "latent_cache_bytes_per_token_layer": 2 * (d.d_c + d.d_rope)}
 
 
 def cache_write_stack(dev, layers: int = 30, reps: int = 3):
