@@ -7,7 +7,7 @@ tokens) into slots 18-20 of a 21-slot ring, then ``videomla_attention`` of those
 prefilled (untimed) by the same cache-write kernel.
 
 Metric: TFLOP/s of the step, counted with the algorithmic flops of the absorbed
-form: per (query, key, head) 2 (d_c + d_rope) + 2 d_c = 832,
+form (App. E): per (query, key, head) 2 (d_c + d_rope) + 2 d_c = 832,
 plus per (query, head) 2 d_nope d_c (absorption) + 2 d_c d_v (W_uv epilogue),
 plus 2 (d_c + d_rope) d_model per written token.
 

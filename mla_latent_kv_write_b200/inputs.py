@@ -11,7 +11,7 @@ Latent KV Cache for Minute-Scale Autoregressive Video Diffusion" (arXiv
 d = 1536, 3-latent-frame chunks) and App. D.2 / Table 4 (d_c = 192,
 d_rope = 32, d_nope = 96, 3D-RoPE pairs (6, 5, 5)).
 
-Distributions (the recipe is restated in the design doc):
+Distributions:
   * activations x, q_nope, q_rope ~ N(0, 1), rounded to bf16 (RNE);
   * weights ~ N(0, 1/fan_in): fan_in = d_model for W_dkv and W_kr, fan_in = d_c
     for the up-projections W_uk and W_uv;

@@ -10,7 +10,7 @@ with the section / equation / table of the paper.  The method reaches exactly
 (up to rounding order) results that have plain definitions, so each function is
 that definition written out in float64 with numpy; matrix products are the only
 library primitive used.  Where the paper is silent, the reading taken is stated
-in the docstring and listed in the design doc.
+in the docstring.
 
 Parity status: every function below is pinned by tests under ``tests/`` that do
 not re-type its formula (printed counts, closed forms, invariants, special cases
