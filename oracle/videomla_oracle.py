@@ -320,3 +320,34 @@ def composite_kv_operator(W_uk: np.ndarray, W_uv: np.ndarray, W_dkv: np.ndarray)
     """M = [W_uk W_dkv ; W_uv W_dkv] ([VideoMLA] §5): the dense-equivalent
     key/value operator, of rank at most d_c by construction."""
     return np.concatenate([W_uk @ W_dkv, W_uv @ W_dkv], axis=0)
+
+
+# ---------------------------------------------------------------------------
+# query path and output projection  ([VideoMLA] §3.1 Eq. 3-4, §3.2 Eq. 6,
+# App. D.2, App. E Eq. 10-11)
+# ---------------------------------------------------------------------------
+
+
+def query_projection(x: np.ndarray, W_dq: np.ndarray, gamma_q: Optional[np.ndarray], eps: float,
+                     W_uq: np.ndarray, W_qr: np.ndarray, n_heads: int):
+    """Per-head queries of new tokens x [..., d]: the query latent
+    c^Q = W_dq x (Eq. 3, W_dq [d_q, d]), RMS-normalised before the
+    up-projections (App. D.2), then q^nope_h = W_uq,h c^Q (Eq. 4,
+    W_uq [H d_nope, d_q]) and the unrotated q^R_h = W_qr,h c^Q (Eq. 6 before
+    RoPE3D, W_qr [H d_rope, d_q]); head h owns row block h of each matrix.
+    Returns (q_nope [..., H, d_nope], q_rope [..., H, d_rope])."""
+    c_q = rms_norm(x @ W_dq.T, gamma_q, eps)
+    q_nope = c_q @ W_uq.T
+    q_rope = c_q @ W_qr.T
+    lead = x.shape[:-1]
+    return (q_nope.reshape(*lead, n_heads, W_uq.shape[0] // n_heads),
+            q_rope.reshape(*lead, n_heads, W_qr.shape[0] // n_heads))
+
+
+def output_projection(o: np.ndarray, W_O: np.ndarray) -> np.ndarray:
+    """Layer output y = sum_h W_O,h o_h for per-head outputs o [..., H, d_v]:
+    W_O [d, H d_v] with column block h applied to head h (the output
+    projection whose per-head slices Eq. 10-11 fold into B_h = W_O,h W_uv,h).
+    Returns y [..., d]."""
+    lead = o.shape[:-2]
+    return o.reshape(*lead, -1) @ W_O.T

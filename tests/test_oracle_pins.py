@@ -487,3 +487,50 @@ def test_sink_pin_catches_sink_after_fifo(monkeypatch):
         m.setattr(O, "window_keys", sink_last)
         out, _ = O.attention_absorbed(**prob, n_sink=1)
     assert np.max(np.abs(out - base_out)) > 1e-6
+
+
+# ---------------------------------------------------------------------------
+# query path and output projection ([VideoMLA] Eq. 3-4, 6, App. D.2, Eq. 10-11)
+# ---------------------------------------------------------------------------
+
+def test_query_projection_brute_force_and_scale_invariance():
+    rng = np.random.default_rng(31)
+    H, d, d_q, d_nope, d_rope = 3, 10, 6, 4, 2
+    x = rng.normal(size=(2, 5, d))
+    W_dq = rng.normal(size=(d_q, d)); g = 1 + 0.1 * rng.normal(size=d_q)
+    W_uq = rng.normal(size=(H * d_nope, d_q)); W_qr = rng.normal(size=(H * d_rope, d_q))
+    eps = 1e-6
+    qn, qr = O.query_projection(x, W_dq, g, eps, W_uq, W_qr, H)
+    for b in range(2):
+        for t in range(5):
+            c = [sum(W_dq[i][k] * x[b, t, k] for k in range(d)) for i in range(d_q)]
+            ms = sum(v * v for v in c) / d_q
+            c = [g[i] * c[i] / math.sqrt(ms + eps) for i in range(d_q)]
+            for h in range(H):
+                for e in range(d_nope):
+                    ref = sum(W_uq[h * d_nope + e][i] * c[i] for i in range(d_q))
+                    assert abs(qn[b, t, h, e] - ref) < 1e-10
+                for e in range(d_rope):
+                    ref = sum(W_qr[h * d_rope + e][i] * c[i] for i in range(d_q))
+                    assert abs(qr[b, t, h, e] - ref) < 1e-10
+    # RMSNorm before the up-projections: scaling a token leaves its queries unchanged
+    qn2, qr2 = O.query_projection(7.5 * x, W_dq, g, 0.0, W_uq, W_qr, H)
+    qn0, qr0 = O.query_projection(x, W_dq, g, 0.0, W_uq, W_qr, H)
+    assert np.max(np.abs(qn2 - qn0)) < 1e-10 and np.max(np.abs(qr2 - qr0)) < 1e-10
+
+
+def test_output_projection_equals_absorbed_value_path():
+    """Eq. 10-11: applying W_O,h to the head output W_uv,h (sum_j p_j c_j) equals
+    applying B_h = W_O,h W_uv,h to the weighted latent sum; and a brute force."""
+    rng = np.random.default_rng(32)
+    H, d_v, d_c, d = 3, 4, 5, 7
+    lat = rng.normal(size=(2, H, d_c))                  # sum_j p_j c_j per head
+    W_uv = rng.normal(size=(H * d_v, d_c)); W_O = rng.normal(size=(d, H * d_v))
+    o = np.stack([lat[:, h] @ W_uv[h * d_v:(h + 1) * d_v].T for h in range(H)], axis=1)   # [2, H, d_v]
+    y = O.output_projection(o, W_O)
+    y_abs = sum(lat[:, h] @ (W_O[:, h * d_v:(h + 1) * d_v] @ W_uv[h * d_v:(h + 1) * d_v]).T for h in range(H))
+    assert np.max(np.abs(y - y_abs)) < 1e-10
+    for n in range(2):
+        for r in range(d):
+            ref = sum(W_O[r][h * d_v + e] * o[n, h, e] for h in range(H) for e in range(d_v))
+            assert abs(y[n, r] - ref) < 1e-10
