@@ -182,6 +182,45 @@ int videomla_attention_sink(const videomla_dims* dims, const void* q_nope, const
                             size_t workspace_bytes, void* stream);
 
 /*
+ * Bytes of the workspace videomla_query_projection needs: the fp32 query latent
+ * and its normalised bf16 copy, for batch * n_tok tokens.  0 for invalid arguments.
+ */
+size_t videomla_query_projection_workspace_size(const videomla_dims* dims, int d_q, int batch, int n_tok);
+
+/*
+ * videomla_query_projection -- per-head queries of new tokens ("VideoMLA",
+ * Sec. 3.1 Eq. 3-4, Sec. 3.2 Eq. 6, App. D.2):
+ *   c^Q = W_dq x (fp32), RMSNorm with gain gamma_q and dims->rms_eps (App. D.2),
+ *   q_nope = W_uq c^Q and q_rope = W_qr c^Q (unrotated; videomla_attention rotates it).
+ *   x       [batch, n_tok, d_model] bf16
+ *   W_dq    [d_q, d_model] bf16; gamma_q [d_q] fp32 or NULL (unit gain)
+ *   W_uq    [n_heads * d_nope, d_q] bf16, W_qr [n_heads * d_rope, d_q] bf16
+ *   q_nope  [batch, n_tok, n_heads, d_nope] bf16, q_rope [batch, n_tok, n_heads, d_rope] bf16
+ *   workspace  at least videomla_query_projection_workspace_size() bytes, 16-byte aligned.
+ * Three tcgen05 GEMM launches and one row-normalisation launch on ``stream``.
+ * Errors: EINVAL (null, d_q or d_model not a multiple of 64, n_heads * d_nope or
+ * n_heads * d_rope not a multiple of 8, small workspace, misaligned), ECUDA.
+ */
+int videomla_query_projection(const videomla_dims* dims, int d_q, const void* x, int batch, int n_tok,
+                              const void* W_dq, const float* gamma_q, const void* W_uq, const void* W_qr,
+                              void* q_nope, void* q_rope, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/*
+ * videomla_output_projection -- layer output y = W_O [o_1 .. o_H] of the per-head
+ * attention outputs (the output projection whose per-head slices W_O,h Eq. 10-11
+ * fold into B_h = W_O,h W_uv,h; applied after W_uv here, which costs fewer flops
+ * than B_h when d_c > d_v).
+ *   o    [batch, n_query, n_heads, d_v] bf16 (videomla_attention's out)
+ *   W_O  [d_model, n_heads * d_v] bf16
+ *   y    [batch, n_query, d_model] bf16
+ * One tcgen05 GEMM launch on ``stream``.
+ * Errors: EINVAL (null, n_heads * d_v not a multiple of 64, misaligned), ECUDA.
+ */
+int videomla_output_projection(const videomla_dims* dims, const void* o, int batch, int n_query, const void* W_O,
+                               void* y, void* stream);
+
+/*
  * Bytes of the library's built-in scratch array used by
  * videomla_attention_static_workspace (16 MiB per device that loads the library).
  */

@@ -13,6 +13,7 @@
 #include "../../include/videomla.h"
 #include "attention.cuh"
 #include "cache_write.cuh"
+#include "gemm.cuh"
 #include "ptx.cuh"
 
 namespace {
@@ -336,6 +337,50 @@ int run_attention(const videomla_dims* d, const void* q_nope, const void* q_rope
     return launch_status(kern, C::SMEM);
 }
 
+
+// ----------------------------------------------------------------------------
+// projections: C [M, N] = A [M, K] . B [N, K]^T
+// ----------------------------------------------------------------------------
+template <int BN, bool F32OUT>
+int run_gemm(const void* A, const void* B, int M, int N, int K, void* Cmat, int ldc, cudaStream_t st) {
+    using C = vmla::GemmCfg<BN, F32OUT>;
+    CUtensorMap ta, tb;
+    {
+        const uint64_t dims[2] = {uint64_t(K), uint64_t(M)};
+        const uint64_t str[1] = {uint64_t(K) * 2};
+        const uint32_t box[2] = {64, uint32_t(C::BM)};
+        if (!make_map(&ta, A, 2, dims, str, box, 128)) return VIDEOMLA_ECUDA;
+    }
+    {
+        const uint64_t dims[2] = {uint64_t(K), uint64_t(N)};
+        const uint64_t str[1] = {uint64_t(K) * 2};
+        const uint32_t box[2] = {64, uint32_t(BN)};
+        if (!make_map(&tb, B, 2, dims, str, box, 128)) return VIDEOMLA_ECUDA;
+    }
+    auto kern = vmla::gemm_kernel<C>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+        return VIDEOMLA_ECUDA;
+    vmla::GemmParams p;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.C = Cmat;
+    p.ldc = ldc;
+    p.timeout_ns = g_timeout_ns.load();
+    dim3 grid((M + C::BM - 1) / C::BM, (N + BN - 1) / BN);
+    kern<<<grid, C::THREADS, C::SMEM, st>>>(ta, tb, p);
+    return launch_status(kern, C::SMEM);
+}
+
+// bf16 C unless f32out; 256-column tiles when they divide N, else 128.
+int gemm(const void* A, const void* B, int M, int N, int K, void* Cmat, int ldc, bool f32out, cudaStream_t st) {
+    if (N % 256 == 0)
+        return f32out ? run_gemm<256, true>(A, B, M, N, K, Cmat, ldc, st) : run_gemm<256, false>(A, B, M, N, K, Cmat, ldc, st);
+    return f32out ? run_gemm<128, true>(A, B, M, N, K, Cmat, ldc, st) : run_gemm<128, false>(A, B, M, N, K, Cmat, ldc, st);
+}
+
+size_t align256(size_t n) { return (n + 255) / 256 * 256; }
+
 }  // namespace
 
 extern "C" {
@@ -419,6 +464,48 @@ int videomla_attention(const videomla_dims* dims, const void* q_nope, const void
                        void* out, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
     return videomla_attention_sink(dims, q_nope, q_rope, W_uk, W_uv, cache, window, nullptr, 0, batch, n_query, out,
                                    lse, workspace, workspace_bytes, stream);
+}
+
+size_t videomla_query_projection_workspace_size(const videomla_dims* dims, int d_q, int batch, int n_tok) {
+    if (!dims || d_q <= 0 || batch <= 0 || n_tok <= 0) return 0;
+    const size_t m = size_t(batch) * n_tok;
+    return align256(m * d_q * 4) + m * d_q * 2;
+}
+
+int videomla_query_projection(const videomla_dims* dims, int d_q, const void* x, int batch, int n_tok,
+                              const void* W_dq, const float* gamma_q, const void* W_uq, const void* W_qr,
+                              void* q_nope, void* q_rope, void* workspace, size_t workspace_bytes, void* stream) {
+    if (!basic_dims_ok(dims) || !x || !W_dq || !W_uq || !W_qr || !q_nope || !q_rope || !workspace)
+        return VIDEOMLA_EINVAL;
+    if (d_q <= 0 || d_q % 64 != 0 || dims->d_model % 64 != 0 || batch <= 0 || n_tok <= 0) return VIDEOMLA_EINVAL;
+    const long long M = (long long)batch * n_tok;
+    const long long nq = (long long)dims->n_heads * dims->d_nope, nr = (long long)dims->n_heads * dims->d_rope;
+    if (M > (1ll << 30) || nq % 8 != 0 || nr % 8 != 0 || nq > (1 << 30) || nr > (1 << 30)) return VIDEOMLA_EINVAL;
+    if (workspace_bytes < videomla_query_projection_workspace_size(dims, d_q, batch, n_tok)) return VIDEOMLA_EINVAL;
+    if (!aligned16(x) || !aligned16(W_dq) || !aligned16(W_uq) || !aligned16(W_qr) || !aligned16(q_nope) ||
+        !aligned16(q_rope) || !aligned16(workspace) || !aligned16(gamma_q))
+        return VIDEOMLA_EINVAL;
+    if (int rc = check_device()) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float* cq = static_cast<float*>(workspace);
+    auto* cqn = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(workspace) + align256(size_t(M) * d_q * 4));
+    // c^Q = x W_dq^T (fp32), RMSNorm -> bf16, then the two up-projections
+    if (int rc = gemm(x, W_dq, int(M), d_q, dims->d_model, cq, d_q, true, st)) return rc;
+    vmla::rms_norm_rows_kernel<<<int((M + 7) / 8), 256, 0, st>>>(cq, cqn, gamma_q, int(M), d_q, dims->rms_eps);
+    if (cudaGetLastError() != cudaSuccess) return VIDEOMLA_ECUDA;
+    if (int rc = gemm(cqn, W_uq, int(M), int(nq), d_q, q_nope, int(nq), false, st)) return rc;
+    return gemm(cqn, W_qr, int(M), int(nr), d_q, q_rope, int(nr), false, st);
+}
+
+int videomla_output_projection(const videomla_dims* dims, const void* o, int batch, int n_query, const void* W_O,
+                               void* y, void* stream) {
+    if (!basic_dims_ok(dims) || !o || !W_O || !y || batch <= 0 || n_query <= 0) return VIDEOMLA_EINVAL;
+    const long long M = (long long)batch * n_query;
+    const long long K = (long long)dims->n_heads * dims->d_v;
+    if (M > (1ll << 30) || K % 64 != 0 || K > (1 << 30) || dims->d_model % 8 != 0) return VIDEOMLA_EINVAL;
+    if (!aligned16(o) || !aligned16(W_O) || !aligned16(y)) return VIDEOMLA_EINVAL;
+    if (int rc = check_device()) return rc;
+    return gemm(o, W_O, int(M), dims->d_model, int(K), y, dims->d_model, false, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

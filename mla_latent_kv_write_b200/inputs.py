@@ -43,6 +43,7 @@ class Dims:
     pairs: tuple = (6, 5, 5)
     rope_base: float = 10000.0
     rms_eps: float = 1e-6
+    d_q: int = 768          # query latent width (App. D.2)
 
     @property
     def tokens_per_frame(self) -> int:
@@ -123,6 +124,25 @@ def _normal(gen: torch.Generator, shape, std: float = 1.0) -> torch.Tensor:
     if std != 1.0:
         t = t * std
     return t.to(torch.bfloat16)
+
+
+def projection_weights(dims: Dims, seed: int, random_gamma: bool = False) -> Dict[str, torch.Tensor]:
+    """Random-init query-path and output weights of one layer (CPU tensors):
+    W_dq [d_q, d_model], W_uq [H*d_nope, d_q], W_qr [H*d_rope, d_q],
+    W_O [d_model, H*d_v] in bf16 (N(0, 1/fan_in)); gamma_q [d_q] in fp32."""
+    g = torch.Generator().manual_seed(seed)
+    d, H = dims.d_model, dims.n_heads
+    w = {
+        "W_dq": _normal(g, (dims.d_q, d), d ** -0.5),
+        "W_uq": _normal(g, (H * dims.d_nope, dims.d_q), dims.d_q ** -0.5),
+        "W_qr": _normal(g, (H * dims.d_rope, dims.d_q), dims.d_q ** -0.5),
+        "W_O": _normal(g, (d, H * dims.d_v), (H * dims.d_v) ** -0.5),
+    }
+    if random_gamma:
+        w["gamma_q"] = 1.0 + 0.1 * torch.randn(dims.d_q, generator=g, dtype=torch.float32)
+    else:
+        w["gamma_q"] = torch.ones(dims.d_q, dtype=torch.float32)
+    return w
 
 
 def layer_weights(dims: Dims, seed: int, random_gamma: bool = False) -> Dict[str, torch.Tensor]:

@@ -31,6 +31,9 @@ EXPORTED = (
     "videomla_attention_static_workspace",
     "videomla_attention_sink",
     "videomla_attention_sink_workspace_size",
+    "videomla_query_projection",
+    "videomla_query_projection_workspace_size",
+    "videomla_output_projection",
     "videomla_strerror",
     "videomla_device_status",
     "videomla_set_wait_timeout_ns",
@@ -82,6 +85,13 @@ def load_library() -> ctypes.CDLL:
         lib.videomla_attention_sink.restype = ci
         lib.videomla_attention_sink_workspace_size.argtypes = [ctypes.POINTER(CDims), ctypes.POINTER(CWindow), ci, ci]
         lib.videomla_attention_sink_workspace_size.restype = ctypes.c_size_t
+        lib.videomla_query_projection_workspace_size.argtypes = [ctypes.POINTER(CDims), ci, ci, ci]
+        lib.videomla_query_projection_workspace_size.restype = ctypes.c_size_t
+        lib.videomla_query_projection.argtypes = [ctypes.POINTER(CDims), ci, vp, ci, ci, vp, vp, vp, vp, vp, vp, vp,
+                                                  ctypes.c_size_t, vp]
+        lib.videomla_query_projection.restype = ci
+        lib.videomla_output_projection.argtypes = [ctypes.POINTER(CDims), vp, ci, ci, vp, vp, vp]
+        lib.videomla_output_projection.restype = ci
         lib.videomla_strerror.argtypes = [ci]
         lib.videomla_strerror.restype = ctypes.c_char_p
         lib.videomla_device_status.argtypes = [ci]
@@ -218,6 +228,56 @@ def attention(q_nope: torch.Tensor, q_rope: torch.Tensor, W_uk: torch.Tensor, W_
     if rc != OK:
         raise VideoMLAError(rc, "videomla_attention_sink" if sink is not None else "videomla_attention")
     return (out, lse) if lse is not None else out
+
+
+def query_projection(x: torch.Tensor, W_dq: torch.Tensor, gamma_q: Optional[torch.Tensor], W_uq: torch.Tensor,
+                     W_qr: torch.Tensor, dims: Dims, q_nope: Optional[torch.Tensor] = None,
+                     q_rope: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None, stream=None):
+    """Per-head queries (q_nope [B, n, H, d_nope], unrotated q_rope [B, n, H, d_rope])
+    of the tokens x [B, n, d_model]: query latent, RMSNorm, up-projections."""
+    lib = load_library()
+    B, n = x.shape[0], x.shape[1]
+    H, dq, dev = dims.n_heads, dims.d_q, x.device
+    _check(x, "x", torch.bfloat16, (B, n, dims.d_model))
+    _check(W_dq, "W_dq", torch.bfloat16, (dq, dims.d_model), dev)
+    _check(W_uq, "W_uq", torch.bfloat16, (H * dims.d_nope, dq), dev)
+    _check(W_qr, "W_qr", torch.bfloat16, (H * dims.d_rope, dq), dev)
+    if gamma_q is not None:
+        _check(gamma_q, "gamma_q", torch.float32, (dq,), dev)
+    if q_nope is None:
+        q_nope = torch.empty(B, n, H, dims.d_nope, dtype=torch.bfloat16, device=dev)
+    if q_rope is None:
+        q_rope = torch.empty(B, n, H, dims.d_rope, dtype=torch.bfloat16, device=dev)
+    _check(q_nope, "q_nope", torch.bfloat16, (B, n, H, dims.d_nope), dev)
+    _check(q_rope, "q_rope", torch.bfloat16, (B, n, H, dims.d_rope), dev)
+    cd = c_dims(dims)
+    need = int(lib.videomla_query_projection_workspace_size(ctypes.byref(cd), dq, B, n))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    elif workspace.device != dev or workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace must be a {need}-byte buffer on {dev}")
+    rc = lib.videomla_query_projection(ctypes.byref(cd), dq, _ptr(x), B, n, _ptr(W_dq), _ptr(gamma_q), _ptr(W_uq),
+                                       _ptr(W_qr), _ptr(q_nope), _ptr(q_rope), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _stream(stream))
+    if rc != OK:
+        raise VideoMLAError(rc, "videomla_query_projection")
+    return q_nope, q_rope
+
+
+def output_projection(o: torch.Tensor, W_O: torch.Tensor, dims: Dims, y: Optional[torch.Tensor] = None, stream=None):
+    """Layer output y [B, n, d_model] = W_O [o_1 .. o_H] of per-head outputs o [B, n, H, d_v]."""
+    lib = load_library()
+    B, n, H, dev = o.shape[0], o.shape[1], dims.n_heads, o.device
+    _check(o, "o", torch.bfloat16, (B, n, H, dims.d_v))
+    _check(W_O, "W_O", torch.bfloat16, (dims.d_model, H * dims.d_v), dev)
+    if y is None:
+        y = torch.empty(B, n, dims.d_model, dtype=torch.bfloat16, device=dev)
+    _check(y, "y", torch.bfloat16, (B, n, dims.d_model), dev)
+    cd = c_dims(dims)
+    rc = lib.videomla_output_projection(ctypes.byref(cd), _ptr(o), B, n, _ptr(W_O), _ptr(y), _stream(stream))
+    if rc != OK:
+        raise VideoMLAError(rc, "videomla_output_projection")
+    return y
 
 
 def device_status(reset: bool = False) -> int:

@@ -13,6 +13,7 @@ import torch
 
 from mla_latent_kv_write_b200 import inputs as I
 from mla_latent_kv_write_b200 import videomla as V
+from oracle import videomla_oracle as O
 from tests.common import (check_attention, check_cache, check_lse, f64, oracle_attention, oracle_cache,
                           sample_rows, to_bf16)
 
@@ -212,3 +213,85 @@ def test_rolling_chain_40_steps():
         ref_out, _ = oracle_attention(dims, q, w, to_bf16(ref_cache), wl.slots, rw["oldest"], rw["n_valid"], rows)
         check_attention(f64(out.cpu())[:, rows], ref_out, f"step {step}")
     assert V.device_status(reset=True) == V.OK
+
+
+# ---------------------------------------------------------------------------
+# query path, output projection and the whole layer ([VideoMLA] Eq. 3-4, 6,
+# App. D.2, Eq. 10-11)
+# ---------------------------------------------------------------------------
+
+# Tolerances: q passes two bf16 roundings (the normalised query latent and q
+# itself, each of RMS relative size ~1e-3; measured 2.3e-3 together); y one
+# rounding (measured 1.7e-3); the layer chain adds the attention's own error.
+Q_NORM_REL, Y_NORM_REL = 4e-3, 3e-3
+LAYER_NORM_REL = 8e-3   # q rounding + attention (<= 5e-3) + y rounding
+
+
+def _norm_rel(got, ref):
+    return float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
+
+
+@pytest.mark.parametrize("dims,n_tok,B,rows", [
+    (I.TINY, 144, 2, None),
+    (I.WAN, 4680, 1, "sample"),
+])
+def test_query_projection(dims, n_tok, B, rows):
+    pw = I.projection_weights(dims, 610, random_gamma=True)
+    x = I.tokens(dims, B, n_tok, 611)
+    d = _dev(pw)
+    qn, qr = V.query_projection(x.to(DEV), d["W_dq"], d["gamma_q"], d["W_uq"], d["W_qr"], dims)
+    torch.cuda.synchronize()
+    assert V.device_status(reset=True) == V.OK
+    sel = np.arange(n_tok) if rows is None else sample_rows(n_tok, 64, seed=612)
+    xs = f64(x)[:, sel]
+    ref_n, ref_r = O.query_projection(xs, f64(pw["W_dq"]), f64(pw["gamma_q"]), dims.rms_eps, f64(pw["W_uq"]),
+                                      f64(pw["W_qr"]), dims.n_heads)
+    got_n, got_r = f64(qn.cpu())[:, sel], f64(qr.cpu())[:, sel]
+    en, er = _norm_rel(got_n, ref_n), _norm_rel(got_r, ref_r)
+    print(f"\nquery projection n_tok={n_tok} B={B}: q_nope rel {en:.2e} q_rope rel {er:.2e}")
+    assert en <= Q_NORM_REL and er <= Q_NORM_REL
+
+
+def test_output_projection():
+    dims = I.WAN
+    pw = I.projection_weights(dims, 620)
+    g = torch.Generator().manual_seed(621)
+    o = torch.randn(1, 4680, dims.n_heads, dims.d_v, generator=g).to(torch.bfloat16)
+    y = V.output_projection(o.to(DEV), pw["W_O"].to(DEV), dims)
+    torch.cuda.synchronize()
+    sel = sample_rows(4680, 64, seed=622)
+    ref = O.output_projection(f64(o)[:, sel], f64(pw["W_O"]))
+    e = _norm_rel(f64(y.cpu())[:, sel], ref)
+    print(f"\noutput projection: rel {e:.2e}")
+    assert e <= Y_NORM_REL
+
+
+def test_layer_chain_tiny():
+    """One attention layer step: new chunk x -> cache write and query path ->
+    latent attention over the window -> output projection, against the
+    oracle's fp64 chain on the same bf16 inputs."""
+    dims, B, slots, first, n_new = I.TINY, 2, 5, 3, 2
+    T_f = dims.tokens_per_frame
+    w = I.layer_weights(dims, 630, random_gamma=True)
+    pw = I.projection_weights(dims, 631, random_gamma=True)
+    cache0 = I.latent_cache(dims, B, slots, 632)
+    x = I.tokens(dims, B, n_new * T_f, 633)
+    wd, pd = _dev(w), _dev(pw)
+    cache = cache0.to(DEV).clone()
+    xd = x.to(DEV)
+    V.cache_write(xd, wd["W_dkv"], wd["W_kr"], wd["gamma"], cache, dims, slots, first)
+    qn, qr = V.query_projection(xd, pd["W_dq"], pd["gamma_q"], pd["W_uq"], pd["W_qr"], dims)
+    oldest = (first + n_new) % slots   # window full after the write: oldest = slot after the newest frame
+    o = V.attention(qn, qr, wd["W_uk"], wd["W_uv"], cache, dims, slots, oldest, slots)
+    y = V.output_projection(o, pd["W_O"], dims)
+    torch.cuda.synchronize()
+    assert V.device_status(reset=True) == V.OK
+    ref_cache = oracle_cache(dims, x, w, slots, first, base=f64(cache0).copy())
+    ref_qn, ref_qr = O.query_projection(f64(x), f64(pw["W_dq"]), f64(pw["gamma_q"]), dims.rms_eps,
+                                        f64(pw["W_uq"]), f64(pw["W_qr"]), dims.n_heads)
+    ref_o, _ = O.attention_absorbed(ref_qn, ref_qr, f64(w["W_uk"]), f64(w["W_uv"]), ref_cache, slots, oldest, slots,
+                                    dims.grid_h, dims.grid_w, dims.d_c, dims.rope_base, dims.pairs)
+    ref_y = O.output_projection(ref_o, f64(pw["W_O"]))
+    e = _norm_rel(f64(y.cpu()), ref_y)
+    print(f"\nlayer chain tiny: y rel {e:.2e}")
+    assert e <= LAYER_NORM_REL
