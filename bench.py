@@ -511,7 +511,43 @@ def side_workloads(dev, peak: float):
     res["sweep_attention"] = sweep
     torch.cuda.empty_cache()
     res["dense_mha_library"] = dense_mha_library(dev, d, wl.n_query, wl.slots * d.tokens_per_frame)
+    res["layer_step"] = layer_step(dev, peak)
     return res
+
+
+def layer_step(dev, peak: float):
+    """One whole attention-layer step on the Wan chunk: query path (Eq. 3-4, 6),
+    cache write, latent attention over the 21-frame window, output projection;
+    2 rotating input sets, CUDA events around the four calls."""
+    from mla_latent_kv_write_b200 import videomla as V
+    wl, d = WORKLOAD, WORKLOAD.dims
+    T_f = d.tokens_per_frame
+    M = wl.n_query
+    calls = []
+    for k in range(2):
+        seed = I.seed_for(6, k, 0)
+        w = {n: t.to(dev) for n, t in I.layer_weights(d, seed).items()}
+        pw = {n: t.to(dev) for n, t in I.projection_weights(d, seed + 1).items()}
+        x = I.tokens(d, 1, M, seed + 2).to(dev)
+        cache = I.latent_cache(d, 1, wl.slots, seed + 3).to(dev)
+        qn = torch.empty(1, M, d.n_heads, d.d_nope, dtype=torch.bfloat16, device=dev)
+        qr = torch.empty(1, M, d.n_heads, d.d_rope, dtype=torch.bfloat16, device=dev)
+        o = torch.empty(1, M, d.n_heads, d.d_v, dtype=torch.bfloat16, device=dev)
+        y = torch.empty(1, M, d.d_model, dtype=torch.bfloat16, device=dev)
+
+        def call(w=w, pw=pw, x=x, cache=cache, qn=qn, qr=qr, o=o, y=y):
+            V.query_projection(x, pw["W_dq"], pw["gamma_q"], pw["W_uq"], pw["W_qr"], d, q_nope=qn, q_rope=qr)
+            V.cache_write(x, w["W_dkv"], w["W_kr"], w["gamma"], cache, d, wl.slots, wl.prefill)
+            V.attention(qn, qr, w["W_uk"], w["W_uv"], cache, d, wl.slots, 0, wl.slots, out=o)
+            V.output_projection(o, pw["W_O"], d, y=y)
+        calls.append(call)
+    ms = _time_attention_calls(calls, 10)
+    fl_q = 2.0 * M * (d.d_model * d.d_q + d.d_q * d.n_heads * (d.d_nope + d.d_rope))
+    fl_o = 2.0 * M * d.n_heads * d.d_v * d.d_model
+    fl = fl_q + flops_cache_write(d, 1, M) + flops_attention(d, 1, M, wl.slots * T_f) + fl_o
+    return {"workload": "Wan layer step: query path + cache write of 3 frames + attention over 21 frames "
+                        "+ output projection, 4680 tokens", "ms": ms, "tflops": fl / (ms * 1e-3) / 1e12,
+            "frac": fl / (ms * 1e-3) / 1e12 / peak, "flops": fl, "projection_flops": fl_q + fl_o}
 
 
 def dense_mha_library(dev, d, Nq: int, Nk: int):
