@@ -152,7 +152,6 @@ __global__ void __launch_bounds__(192, 1)
                        const __grid_constant__ CUtensorMap tm_wkr, const CacheWriteParams p) {
     using C = CacheWriteCfg<DC, DR>;
     constexpr int N = C::N;
-    constexpr int GROUPS = N / 8;              // 8-column groups of a row
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BUF);
