@@ -97,30 +97,72 @@ def ncu_traffic(kernel: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+    """SM clock, power and clock-event (throttle) reasons of this rank's GPU while
+    the timed region runs: NVML read every 10 ms from a thread (device found by
+    its PCI bus id, so CUDA_VISIBLE_DEVICES cannot point it at another GPU), or
+    nvidia-smi every 200 ms if NVML is unavailable.  Reads only."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASON_BITS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+                   ("sw_power_cap", 0x4))
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
         self.path = None
+        self.rows = []
+        self.thread = None
+        self.stop = None
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.index)
+        bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+        return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
 
     def __enter__(self):
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except (OSError, ValueError):
-            self.proc = None
-        time.sleep(0.3)
+            nv, h = self._nvml_handle()
+            max_sm = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            self.stop = threading.Event()
+
+            def run():
+                while not self.stop.is_set():
+                    try:
+                        sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                        pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                        rs = int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+                        self.rows.append((sm, max_sm, pw, rs))
+                    except Exception:
+                        pass
+                    self.stop.wait(0.01)
+            self.thread = threading.Thread(target=run, daemon=True)
+            self.thread.start()
+            self.source = "nvml, 10 ms"
+        except Exception:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                     "--format=csv,noheader,nounits", "-lms", "200"],
+                    stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                self.source = "nvidia-smi, 200 ms"
+            except (OSError, ValueError):
+                self.proc = None
+            time.sleep(0.3)
         return self
 
     def __exit__(self, *exc):
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=2)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -129,26 +171,29 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        if self.proc is None or not self.path or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        names = tuple(n for n, _ in self.REASON_BITS)
         rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4], parts[5:9]))
-                except ValueError:
-                    continue
-        os.unlink(self.path)
+        if self.thread is not None:
+            for sm, mx, pw, rs in self.rows:
+                rows.append((sm, mx, pw, [("active" if rs & bit else "not active") for _, bit in self.REASON_BITS]))
+        elif self.proc is not None and self.path and os.path.exists(self.path):
+            with open(self.path) as f:
+                for line in f:
+                    parts = [x.strip() for x in line.split(",")]
+                    if len(parts) < 9:
+                        continue
+                    try:
+                        rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+                    except ValueError:
+                        continue
+            os.unlink(self.path)
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "source": self.source}
         loaded = [r for r in rows if r[2] > 200.0] or rows
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[4]) if v.lower() == "active"})
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3]) if v.lower() == "active"})
         return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
-                "power_w_max": max(r[2] for r in rows), "samples": len(loaded), "reasons": reasons}
+                "power_w_max": max(r[2] for r in rows), "samples": len(loaded), "reasons": reasons,
+                "source": self.source}
 
 
 def dist_setup(backend: str = "nccl"):
