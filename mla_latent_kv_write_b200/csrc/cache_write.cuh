@@ -47,7 +47,8 @@ struct CacheWriteCfg {
     static constexpr int BKK = 64;                    // K elements per stage (one 128-B swizzle row)
     static constexpr int N_MMA = N <= 256 ? 1 : 2;    // MMA column chunks
     static constexpr int N_CHUNK = N / N_MMA;
-    static constexpr int NS = N <= 256 ? 4 : 3;       // pipeline stages
+    // pipeline stages: as many as fit (the bytes in flight per SM set its streaming rate)
+    static constexpr int NS = N <= 256 ? ((BM * BKK * 2 + N * BKK * 2) * 5 + 2048 + DC * 4 <= 232448 ? 5 : 4) : 3;
     static constexpr int X_BYTES = BM * BKK * 2;
     static constexpr int W_BYTES = N * BKK * 2;
     static constexpr int STAGE = X_BYTES + W_BYTES;
