@@ -13,13 +13,13 @@
 //   warps 2-5  epilogue.  After a cluster barrier (every CTA's MMAs are done,
 //              so every CTA's pipeline stages are free) each thread copies one
 //              TMEM lane (token row) of its fp32 partial into local shared
-//              memory; one thread then ships each peer the contiguous block of
-//              the rows that peer owns (rows [128 r / ksplit, 128 (r+1) / ksplit)
-//              belong to rank r) with one bulk shared-to-shared copy completing
-//              on the peer's mbarrier.  Each owner sums the ksplit partials of its
-//              rows, one warp per row (lane l holds columns 8l .. 8l+7), reduces
-//              the row's sum of squares with warp shuffles, applies RMSNorm and
-//              writes the row as 16-byte bf16 stores.
+//              memory; each warp then ships its 32 rows to the peers that own
+//              them (rows [128 r / ksplit, 128 (r+1) / ksplit) belong to rank r)
+//              with bulk shared-to-shared copies completing on the peer's
+//              mbarrier.
+//   all warps  each owner sums the ksplit partials of its rows (a quad of
+//              threads per row), reduces the row's sum of squares with warp
+//              shuffles, applies RMSNorm and writes the row as 16-byte bf16 stores.
 #pragma once
 
 #include "ptx.cuh"
@@ -292,23 +292,27 @@ __global__ void __launch_bounds__(192, 1)
             }
         }
         fence_proxy_async_smem();  // the bulk copies read part through the async proxy
-    }
-    // every thread of the CTA: all of ``part`` is written before anyone reads or ships it
-    __syncthreads();
-    if (warp >= 2) {
-        // (b) ship each peer the contiguous block of its rows: one bulk copy per peer
-        if (warp == 2 && lane == 0 && p.ksplit > 1) {
+        __syncwarp();
+        // (b) this warp's 32 rows go to the peers that own them as soon as they are
+        // written (one bulk shared-to-shared copy per owner), overlapping the other
+        // warps' TMEM reads; the copies complete on the owner's mbarrier
+        if (lane == 0 && p.ksplit > 1) {
             for (int k = 0; k < p.ksplit; ++k) {
                 if (k == int(rank)) continue;
                 const int lo = (C::BM * k) / p.ksplit, hi = (C::BM * (k + 1)) / p.ksplit;
+                const int a = max(quarter * 32, lo), e = min(quarter * 32 + 32, hi);
+                if (a >= e) continue;
                 const int slot = int(rank) < k ? int(rank) : int(rank) - 1;
-                const uint32_t dst = mapa_shared(smem_u32(rbuf + slot * rows_max * C::RED_STRIDE), uint32_t(k));
-                bulk_copy_to_peer(dst, smem_u32(part + lo * C::RED_STRIDE), uint32_t((hi - lo) * C::RED_STRIDE * 4),
+                const uint32_t dst =
+                    mapa_shared(smem_u32(rbuf + (slot * rows_max + (a - lo)) * C::RED_STRIDE), uint32_t(k));
+                bulk_copy_to_peer(dst, smem_u32(part + a * C::RED_STRIDE), uint32_t((e - a) * C::RED_STRIDE * 4),
                                   mapa_shared(smem_u32(recv), uint32_t(k)));
             }
             bulk_commit();
         }
     }
+    // every thread of the CTA: all of ``part`` is written before anyone reads its own rows
+    __syncthreads();
 
     // (c) all 192 threads: sum the ksplit partials of this CTA's rows, RMSNorm, bf16 rows
     const bool got = p.ksplit == 1 || __all_sync(0xffffffffu, mbar_wait(recv, 0, ab, p.timeout_ns, 4));
@@ -321,7 +325,7 @@ __global__ void __launch_bounds__(192, 1)
         default: cw_finish_rows<DC, DR, 4>(p, part, rbuf, gs, rows_max, r_lo, r_hi, row0, b, store); break;
     }
     // our outgoing copies must have read ``part`` before this CTA exits
-    if (warp == 2 && lane == 0 && p.ksplit > 1) bulk_wait_read();
+    if (warp >= 2 && lane == 0 && p.ksplit > 1) bulk_wait_read();
 
     tc_fence_before();
     __syncthreads();
