@@ -114,6 +114,19 @@ int videomla_cache_write(const videomla_dims* dims, const void* x, int batch, in
 size_t videomla_attention_workspace_size(const videomla_dims* dims, const videomla_window* window, int batch);
 
 /*
+ * Bytes of a workspace that also holds the split-KV partials of the split the
+ * library prefers for this call: when the (query tile, head, batch) units do not
+ * fill the GPU's SMs in whole waves, the key tiles of each unit are shared by up
+ * to 4 CTAs, each storing an unnormalised partial (fp32 O plus the per-row max
+ * and sum) that the last of them merges.  A workspace between
+ * videomla_attention_workspace_size() (or the sink variant's) and this size makes
+ * the call use the largest split that fits; results agree to rounding.
+ * 0 for invalid arguments.
+ */
+size_t videomla_attention_workspace_size_split(const videomla_dims* dims, const videomla_window* window, int n_sink,
+                                               int batch, int n_query);
+
+/*
  * videomla_attention -- latent attention of the newest n_query tokens of the
  * window over all n_valid * T_f keys of the window (no mask inside it).
  *   q_nope [batch, n_query, n_heads, d_nope] bf16: per-head content queries (Eq. 4).
@@ -129,8 +142,9 @@ size_t videomla_attention_workspace_size(const videomla_dims* dims, const videom
  *   workspace  device scratch of at least videomla_attention_workspace_size()
  *          bytes, 16-byte aligned, owned by the caller; its contents on entry do
  *          not matter and are overwritten (the window's rotated RoPE keys,
- *          App. D.5: rotation applied when the active window is formed).  Calls
- *          that run concurrently need distinct workspaces.
+ *          App. D.5: rotation applied when the active window is formed; with
+ *          videomla_attention_workspace_size_split() bytes also the split-KV
+ *          partials).  Calls that run concurrently need distinct workspaces.
  * Two launches on ``stream``: the window pre-pass, then the attention kernel.
  * Arithmetic: tcgen05 tensor cores with fp32 accumulation; the latent part of
  * the scores uses bf16 operands (q_abs rounded to bf16), the RoPE part fp16

@@ -45,7 +45,15 @@ struct AttnParams {
     int seg_start[3], seg_len[3];
     int n_sink;                    // sink frames (local t = 0 .. n_sink-1; FIFO frames follow)
     int ws_rows;                   // rotated-key workspace rows per batch element: (slots + n_sink) T_f
-    int n_kt;                      // key tiles
+    int n_kt;                      // key tiles of the whole window
+    // split-KV: the key tiles of one (query tile, head, batch) unit are split over
+    // n_split CTAs of tiles_per_split tiles; each writes its unnormalised O and
+    // per-row (max, sum) to part_o / part_ml, and the last of them to arrive
+    // (counters, zeroed by the window pre-pass) merges and finishes the unit
+    int n_split, tiles_per_split, n_units;
+    float* part_o;                 // [n_units * n_split, BM, d_c] fp32
+    float* part_ml;                // [n_units * n_split, BM, 2] fp32: row max (raw score), row sum
+    int* counters;                 // [n_units]
     int q_first;                   // logical window index of query 0
     int n_t, n_h;                  // rope pairs of the t and h axes (w takes the rest)
     float omega[32];               // rope frequency of each pair
@@ -120,6 +128,8 @@ struct AttnCfg {
 
 struct AttnBarriers {
     uint64_t full[4], empty[4];
+    uint64_t part_done, last_known;  // split-KV: partial stored by every softmax warp / arrival counted
+    int last_flag, skip_epilogue;
     uint64_t q_full, qabs_done, q_ready, s_full, s_free, p_full, pv_done, olat_ready, out_full, drain, drain2;
     uint32_t tmem_base;
     AbortState ab;
@@ -163,6 +173,11 @@ __global__ void __launch_bounds__(256) rope_window_kernel(const __nv_bfloat16* _
                                                           const __nv_bfloat16* __restrict__ sink,
                                                           __half* __restrict__ krot, const AttnParams p, int B) {
     constexpr int W = DC + DR, CH = DR / 8;
+    if (p.n_split > 1) {  // arrival counters of the split-KV attention launched next
+        for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < p.n_units;
+             i += (long long)gridDim.x * blockDim.x)
+            p.counters[i] = 0;
+    }
     const int ring_valid = p.seg_len[0] + p.seg_len[1];
     const int rows_valid = ring_valid + p.seg_len[2];
     const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -211,9 +226,10 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
     auto stage = [&](int s) { return smem + s * C::STAGE; };
 
     const int warp = warp_id(), lane = lane_id();
-    const int h = blockIdx.y, b = blockIdx.z;
+    const int h = blockIdx.y, b = blockIdx.z / p.n_split, split = blockIdx.z % p.n_split;
     const int q0 = blockIdx.x * BM;
-    const int nt = p.n_kt;
+    const int kt0 = split * p.tiles_per_split;                      // first key tile of this split
+    const int nt = min(p.n_kt, kt0 + p.tiles_per_split) - kt0;     // key tiles of this CTA (>= 1)
     const uint64_t to = p.timeout_ns;
 
     if (threadIdx.x == 0) {
@@ -232,6 +248,10 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
         mbar_init(&bar->out_full, 1);
         mbar_init(&bar->drain, 1);
         mbar_init(&bar->drain2, 1);
+        mbar_init(&bar->part_done, C::SM_WARPS);
+        mbar_init(&bar->last_known, 1);
+        bar->last_flag = 0;
+        bar->skip_epilogue = 0;
         ab->flag = 0;
         fence_mbar_init();
     }
@@ -274,7 +294,7 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                 if (!ok) break;
                 if (j < nt) {
                     int run, row, valid;
-                    key_tile<BK>(p, j, run, row, valid);
+                    key_tile<BK>(p, kt0 + j, run, row, valid);
                     mbar_arrive_expect_tx(&bar->full[s], C::STAGE);
                     for (int a = 0; a < C::C_ATOMS; ++a)
                         tma_load_3d(stage(s) + a * C::C_ATOM, &maps.cc[run], &bar->full[s], a * 64, row, b);
@@ -355,7 +375,7 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                 for (int w = 0; ok && w < C::WUV_STAGES; ++w)
                     ok = mbar_wait(&bar->full[(nt + w) % NS], ((nt + w) / NS) & 1, ab, to, 35);
                 ok = ok && mbar_wait(&bar->olat_ready, 0, ab, to, 36);
-                if (ok) {
+                if (ok && !*reinterpret_cast<volatile int*>(&bar->skip_epilogue)) {
                     tc_fence_after();
                     constexpr uint32_t id_o = idesc_bf16_f32(128, DV, false, false);
                     const uint32_t ao = smem_u32(C::QS ? qreg : stage((nt + 1) % NS));
@@ -505,7 +525,7 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
             if (lane == 0) mbar_arrive(&bar->s_free);
 
             int run, row, valid;
-            key_tile<BK>(p, j, run, row, valid);
+            key_tile<BK>(p, kt0 + j, run, row, valid);
             if (valid < BK) {  // ragged last tile of a run: mask the missing keys
 #pragma unroll
                 for (int c = 0; c < NC; ++c)
@@ -614,23 +634,102 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
         }
 
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar->pv_done, (nt - 1) & 1, ab, to, 44) && !ab->flag);
+        bool last = true;  // this CTA finishes the unit (always, without split-KV)
+        const int r_top = w4 * 32 + half * 16 + (lane >> 2);
+        const int r_bot = r_top + 8;
+        float m_fin[2] = {m_used[0], m_used[1]}, l_fin[2] = {0.f, 0.f}, f_own[2] = {1.f, 1.f};
+        constexpr int MAXS = 8;             // most splits of one unit
+        float f_oth[MAXS][2];               // scale of split s's partial in the merged sum
         if (ok) {
             tc_fence_after();
-            float inv[2], lt[2];
 #pragma unroll
             for (int k = 0; k < 2; ++k) {
-                lt[k] = l_part[k];
-                lt[k] += __shfl_xor_sync(0xffffffffu, lt[k], 1);
-                lt[k] += __shfl_xor_sync(0xffffffffu, lt[k], 2);
-                inv[k] = 1.0f / lt[k];
+                l_fin[k] = l_part[k];
+                l_fin[k] += __shfl_xor_sync(0xffffffffu, l_fin[k], 1);
+                l_fin[k] += __shfl_xor_sync(0xffffffffu, l_fin[k], 2);
             }
+        }
+        const int unit = (b * p.H + h) * int(gridDim.x) + int(blockIdx.x);
+        if (ok && p.n_split > 1) {
+            // (1) this split's unnormalised O and (max, sum) -> workspace
+            const size_t slot = size_t(unit) * p.n_split + split;
+            float* po = p.part_o + slot * (BM * DC);
+#pragma unroll 1
+            for (int c32 = 0; c32 < DC / 32; c32 += 2) {
+                uint32_t o[32];
+                const bool full = c32 + 2 <= DC / 32;
+                if (full) {
+                    tmem_ld_16x256b_x8(tb + C::O_COL + c32 * 32, o);
+                } else {
+                    tmem_ld_16x256b_x4(tb + C::O_COL + c32 * 32, *reinterpret_cast<uint32_t(*)[16]>(o));
+                }
+                tmem_wait_ld();
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    if (!full && k >= 4) break;
+                    const int col = c32 * 32 + 8 * k + 2 * quad;
+                    *reinterpret_cast<float2*>(po + r_top * DC + col) =
+                        make_float2(__uint_as_float(o[4 * k]), __uint_as_float(o[4 * k + 1]));
+                    *reinterpret_cast<float2*>(po + r_bot * DC + col) =
+                        make_float2(__uint_as_float(o[4 * k + 2]), __uint_as_float(o[4 * k + 3]));
+                }
+            }
+            if (quad == 0) {
+                *reinterpret_cast<float2*>(p.part_ml + (slot * BM + r_top) * 2) = make_float2(m_used[0], l_fin[0]);
+                *reinterpret_cast<float2*>(p.part_ml + (slot * BM + r_bot) * 2) = make_float2(m_used[1], l_fin[1]);
+            }
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar->part_done);
+            // (2) once all 8 warps have stored, count this split; the last to arrive merges
+            if (warp == 2) {
+                const bool stored = __all_sync(0xffffffffu, mbar_wait(&bar->part_done, 0, ab, to, 46));
+                if (lane == 0) {
+                    const int prev = stored ? atomicAdd(&p.counters[unit], 1) : -1;
+                    bar->last_flag = prev == p.n_split - 1;
+                    mbar_arrive(&bar->last_known);
+                }
+                __syncwarp();
+            }
+            ok = __all_sync(0xffffffffu, mbar_wait(&bar->last_known, 0, ab, to, 47) && !ab->flag);
+            last = ok && *reinterpret_cast<volatile int*>(&bar->last_flag) != 0;
+            if (last) {
+                __threadfence();
+                // merged row max and sum over the splits (each split's m is a raw score)
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const int r = k ? r_bot : r_top;
+                    float mt = m_used[k];
+                    for (int sp = 0; sp < p.n_split; ++sp)
+                        if (sp != split)
+                            mt = fmaxf(mt, __ldcg(p.part_ml + ((size_t(unit) * p.n_split + sp) * BM + r) * 2));
+                    f_own[k] = ex2((m_used[k] - mt) * sl);
+                    float lsum = l_fin[k] * f_own[k];
+#pragma unroll
+                    for (int sp = 0; sp < MAXS; ++sp) {
+                        f_oth[sp][k] = 0.f;
+                        if (sp < p.n_split && sp != split) {
+                            const float2 ml = __ldcg(reinterpret_cast<const float2*>(
+                                p.part_ml + ((size_t(unit) * p.n_split + sp) * BM + r) * 2));
+                            f_oth[sp][k] = ex2((ml.x - mt) * sl);
+                            lsum += ml.y * f_oth[sp][k];
+                        }
+                    }
+                    m_fin[k] = mt;
+                    l_fin[k] = lsum;
+                }
+            }
+        }
+        if (ok && last) {
+            float inv[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) inv[k] = 1.0f / l_fin[k];
             // O_lat = O / l, K-major SW128: hi + lo bf16 parts in stages (nt+1) % NS and
             // (nt+2) % NS, or (QS) one bf16 part in the Q region; all are idle: every S and
-            // PV MMA has completed
+            // PV MMA has completed.  With split-KV, O is this split's O scaled to the merged
+            // max plus every other split's stored O, likewise scaled.
             uint8_t* ol = C::QS ? qreg : stage((nt + 1) % NS);
             uint8_t* ol2 = stage((nt + 2) % NS);
-            const int r_top = w4 * 32 + half * 16 + (lane >> 2);
-            const int r_bot = r_top + 8;
 #pragma unroll 1
             for (int c32 = 0; c32 < DC / 32; c32 += 2) {  // 64 columns, or the last 32
                 uint32_t o[32];
@@ -641,6 +740,38 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                     tmem_ld_16x256b_x4(tb + C::O_COL + c32 * 32, *reinterpret_cast<uint32_t(*)[16]>(o));
                 }
                 tmem_wait_ld();
+                float v[32];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    v[4 * k + 0] = __uint_as_float(o[4 * k + 0]) * f_own[0];
+                    v[4 * k + 1] = __uint_as_float(o[4 * k + 1]) * f_own[0];
+                    v[4 * k + 2] = __uint_as_float(o[4 * k + 2]) * f_own[1];
+                    v[4 * k + 3] = __uint_as_float(o[4 * k + 3]) * f_own[1];
+                }
+                if (p.n_split > 1) {
+                    for (int sp = 0; sp < p.n_split; ++sp) {
+                        if (sp == split) continue;
+                        const float* ps = p.part_o + (size_t(unit) * p.n_split + sp) * (BM * DC);
+                        float fa = 0.f, fb = 0.f;
+#pragma unroll
+                        for (int q = 0; q < MAXS; ++q)
+                            if (q == sp) {
+                                fa = f_oth[q][0];
+                                fb = f_oth[q][1];
+                            }
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            if (!full && k >= 4) break;
+                            const int col = c32 * 32 + 8 * k + 2 * quad;
+                            const float2 t = __ldcg(reinterpret_cast<const float2*>(ps + r_top * DC + col));
+                            const float2 u = __ldcg(reinterpret_cast<const float2*>(ps + r_bot * DC + col));
+                            v[4 * k + 0] = fmaf(t.x, fa, v[4 * k + 0]);
+                            v[4 * k + 1] = fmaf(t.y, fa, v[4 * k + 1]);
+                            v[4 * k + 2] = fmaf(u.x, fb, v[4 * k + 2]);
+                            v[4 * k + 3] = fmaf(u.y, fb, v[4 * k + 3]);
+                        }
+                    }
+                }
                 const int cc = c32 / 2;
                 const int off_top = cc * C::OLAT_ATOM + r_top * 128 + 4 * quad;
                 const int off_bot = cc * C::OLAT_ATOM + r_bot * 128 + 4 * quad;
@@ -648,17 +779,15 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                 for (int k = 0; k < 8; ++k) {
                     if (!full && k >= 4) break;
                     uint32_t hi, lo;
-                    split_bf16(__uint_as_float(o[4 * k]) * inv[0], __uint_as_float(o[4 * k + 1]) * inv[0], hi, lo);
+                    split_bf16(v[4 * k] * inv[0], v[4 * k + 1] * inv[0], hi, lo);
                     const int ot = off_top + ((k ^ (r_top & 7)) << 4);
-                    *reinterpret_cast<uint32_t*>(ol + ot) = C::QS ? pack_bf16(__uint_as_float(o[4 * k]) * inv[0],
-                                                                              __uint_as_float(o[4 * k + 1]) * inv[0])
-                                                                  : hi;
+                    *reinterpret_cast<uint32_t*>(ol + ot) =
+                        C::QS ? pack_bf16(v[4 * k] * inv[0], v[4 * k + 1] * inv[0]) : hi;
                     if constexpr (!C::QS) *reinterpret_cast<uint32_t*>(ol2 + ot) = lo;
-                    split_bf16(__uint_as_float(o[4 * k + 2]) * inv[1], __uint_as_float(o[4 * k + 3]) * inv[1], hi, lo);
+                    split_bf16(v[4 * k + 2] * inv[1], v[4 * k + 3] * inv[1], hi, lo);
                     const int ob = off_bot + ((k ^ (r_bot & 7)) << 4);
-                    *reinterpret_cast<uint32_t*>(ol + ob) = C::QS ? pack_bf16(__uint_as_float(o[4 * k + 2]) * inv[1],
-                                                                              __uint_as_float(o[4 * k + 3]) * inv[1])
-                                                                  : hi;
+                    *reinterpret_cast<uint32_t*>(ol + ob) =
+                        C::QS ? pack_bf16(v[4 * k + 2] * inv[1], v[4 * k + 3] * inv[1]) : hi;
                     if constexpr (!C::QS) *reinterpret_cast<uint32_t*>(ol2 + ob) = lo;
                 }
             }
@@ -672,7 +801,7 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                 for (int k = 0; k < 2; ++k) {
                     const int i = q0 + r_top + 8 * k;
                     if (i < p.Nq)
-                        p.lse[(size_t(b) * p.Nq + i) * p.H + h] = (m_used[k] * sl + __log2f(lt[k])) * 0.69314718055994531f;
+                        p.lse[(size_t(b) * p.Nq + i) * p.H + h] = (m_fin[k] * sl + __log2f(l_fin[k])) * 0.69314718055994531f;
                 }
             }
 
@@ -697,6 +826,12 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                         for (int e = 0; e < 4; ++e) d4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
                     }
                 }
+            }
+        } else if (ok) {
+            // not the last split of this unit: the last one writes its output
+            if (lane == 0) {
+                bar->skip_epilogue = 1;
+                mbar_arrive(&bar->olat_ready);
             }
         }
     }

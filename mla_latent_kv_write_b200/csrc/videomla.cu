@@ -73,6 +73,7 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, 
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t align256(size_t n) { return (n + 255) / 256 * 256; }
 
 // sm_100 check, cached per device.
 int check_device() {
@@ -239,10 +240,39 @@ void window_runs(const videomla_window* win, int T_f, int seg_start[3], int seg_
     }
 }
 
+// Split-KV of the attention: how many CTAs share the key tiles of one (query
+// tile, head, batch) unit.  One CTA per SM; cost in key-tile times: the waves
+// times the tiles per CTA (+2 for writing a partial), plus the merge of the
+// other partials by the last CTA (1.5 per split).  At most 4 splits.
+int preferred_split(int units, int n_kt, int batch) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+    int best = 1;
+    double best_cost = 0;
+    for (int s = 1; s <= 4 && s <= n_kt && (long long)batch * s <= 65535; ++s) {
+        const int tps = (n_kt + s - 1) / s;
+        const int se = (n_kt + tps - 1) / tps;
+        if (se != s) continue;
+        const long long waves = ((long long)units * s + sms - 1) / sms;
+        const double cost = double(waves) * (tps + (s > 1 ? 2 : 0)) + 1.5 * (s - 1);
+        if (s == 1 || cost < best_cost) {
+            best = s;
+            best_cost = cost;
+        }
+    }
+    return best;
+}
+
+size_t split_part_bytes(int units, int split, int d_c) {  // partial O + (max, sum) per row + counters
+    if (split <= 1) return 0;
+    return size_t(units) * split * (128 * size_t(d_c) * 4 + 128 * 2 * 4) + align256(size_t(units) * 4);
+}
+
 template <int DC, int DR, int DN, int DV>
 int run_attention(const videomla_dims* d, const void* q_nope, const void* q_rope, const void* W_uk, const void* W_uv,
                   const void* cache, const videomla_window* win, const void* sink, int n_sink, int B, int Nq,
-                  void* out, float* lse, void* workspace, cudaStream_t st) {
+                  void* out, float* lse, void* workspace, size_t workspace_bytes, cudaStream_t st) {
     using C = vmla::AttnCfg<DC, DR, DN, DV>;
     const int T_f = d->grid_h * d->grid_w;
     const int H = d->n_heads;
@@ -262,6 +292,20 @@ int run_attention(const videomla_dims* d, const void* q_nope, const void* q_rope
     p.ws_rows = (win->slots + n_sink) * T_f;
     p.n_kt = 0;
     for (int r = 0; r < 3; ++r) p.n_kt += (p.seg_len[r] + C::BK - 1) / C::BK;
+    {
+        // split-KV, as far as the workspace holds the partials
+        const int units = (Nq + C::BM - 1) / C::BM * H * B;
+        const size_t rope_bytes = align256(size_t(B) * p.ws_rows * DR * 2);
+        int sp = preferred_split(units, p.n_kt, B);
+        while (sp > 1 && rope_bytes + split_part_bytes(units, sp, DC) > workspace_bytes) --sp;
+        p.tiles_per_split = (p.n_kt + sp - 1) / sp;
+        p.n_split = (p.n_kt + p.tiles_per_split - 1) / p.tiles_per_split;
+        p.n_units = units;
+        uint8_t* wsb = static_cast<uint8_t*>(workspace);
+        p.part_o = reinterpret_cast<float*>(wsb + rope_bytes);
+        p.part_ml = p.part_o + size_t(units) * p.n_split * 128 * DC;
+        p.counters = reinterpret_cast<int*>(p.part_ml + size_t(units) * p.n_split * 128 * 2);
+    }
     p.q_first = (n_sink + win->n_valid) * T_f - Nq;
     p.n_t = d->pairs_t;
     p.n_h = d->pairs_h;
@@ -332,7 +376,7 @@ int run_attention(const videomla_dims* d, const void* q_nope, const void* q_rope
     auto kern = vmla::attention_kernel<C>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
         return VIDEOMLA_ECUDA;
-    dim3 grid((Nq + C::BM - 1) / C::BM, H, B);
+    dim3 grid((Nq + C::BM - 1) / C::BM, H, B * p.n_split);
     kern<<<grid, C::THREADS, C::SMEM, st>>>(maps, p);
     return launch_status(kern, C::SMEM);
 }
@@ -379,7 +423,6 @@ int gemm(const void* A, const void* B, int M, int N, int K, void* Cmat, int ldc,
     return f32out ? run_gemm<128, true>(A, B, M, N, K, Cmat, ldc, st) : run_gemm<128, false>(A, B, M, N, K, Cmat, ldc, st);
 }
 
-size_t align256(size_t n) { return (n + 255) / 256 * 256; }
 
 }  // namespace
 
@@ -425,6 +468,25 @@ size_t videomla_attention_workspace_size(const videomla_dims* dims, const videom
     return videomla_attention_sink_workspace_size(dims, window, 0, batch);
 }
 
+size_t videomla_attention_workspace_size_split(const videomla_dims* dims, const videomla_window* window, int n_sink,
+                                               int batch, int n_query) {
+    const size_t rope = videomla_attention_sink_workspace_size(dims, window, n_sink, batch);
+    if (rope == 0 || n_query <= 0 || dims->n_heads <= 0) return 0;
+    const int T_f = dims->grid_h * dims->grid_w;
+    const int bk = (dims->d_c + 128 + 64 + (dims->d_c + dims->d_rope) / 2 > 512) ? 64 : 128;  // key tile
+    // key tiles per run, as run_attention counts them
+    videomla_window w = *window;
+    if (w.slots <= 0 || w.n_valid < 1 || w.n_valid > w.slots || w.oldest_slot < 0 || w.oldest_slot >= w.slots)
+        return 0;
+    int seg_start[3], seg_len[3];
+    window_runs(&w, T_f, seg_start, seg_len);
+    seg_len[2] = n_sink * T_f;
+    int n_kt = 0;
+    for (int r = 0; r < 3; ++r) n_kt += (seg_len[r] + bk - 1) / bk;
+    const int units = (n_query + 127) / 128 * dims->n_heads * batch;
+    return align256(rope) + split_part_bytes(units, preferred_split(units, n_kt, batch), dims->d_c);
+}
+
 int videomla_attention_sink(const videomla_dims* dims, const void* q_nope, const void* q_rope, const void* W_uk,
                             const void* W_uv, const void* cache, const videomla_window* window, const void* sink_cache,
                             int n_sink, int batch, int n_query, void* out, float* lse, void* workspace,
@@ -449,7 +511,7 @@ int videomla_attention_sink(const videomla_dims* dims, const void* q_nope, const
 #define VMLA_AT(DC_, DR_, DN_, DV_)                        \
     if (dc == DC_ && dr == DR_ && dn == DN_ && dv == DV_) \
         return run_attention<DC_, DR_, DN_, DV_>(dims, q_nope, q_rope, W_uk, W_uv, cache, &w, sink_cache, n_sink, \
-                                                 batch, n_query, out, lse, workspace, st);
+                                                 batch, n_query, out, lse, workspace, workspace_bytes, st);
     VMLA_AT(192, 32, 96, 128)
     VMLA_AT(192, 16, 112, 128)
     VMLA_AT(192, 64, 64, 128)

@@ -31,6 +31,7 @@ EXPORTED = (
     "videomla_attention_static_workspace",
     "videomla_attention_sink",
     "videomla_attention_sink_workspace_size",
+    "videomla_attention_workspace_size_split",
     "videomla_query_projection",
     "videomla_query_projection_workspace_size",
     "videomla_output_projection",
@@ -85,6 +86,9 @@ def load_library() -> ctypes.CDLL:
         lib.videomla_attention_sink.restype = ci
         lib.videomla_attention_sink_workspace_size.argtypes = [ctypes.POINTER(CDims), ctypes.POINTER(CWindow), ci, ci]
         lib.videomla_attention_sink_workspace_size.restype = ctypes.c_size_t
+        lib.videomla_attention_workspace_size_split.argtypes = [ctypes.POINTER(CDims), ctypes.POINTER(CWindow), ci, ci,
+                                                                ci]
+        lib.videomla_attention_workspace_size_split.restype = ctypes.c_size_t
         lib.videomla_query_projection_workspace_size.argtypes = [ctypes.POINTER(CDims), ci, ci, ci]
         lib.videomla_query_projection_workspace_size.restype = ctypes.c_size_t
         lib.videomla_query_projection.argtypes = [ctypes.POINTER(CDims), ci, vp, ci, ci, vp, vp, vp, vp, vp, vp, vp,
@@ -167,11 +171,16 @@ def cache_write(x: torch.Tensor, W_dkv: torch.Tensor, W_kr: torch.Tensor, gamma:
     return cache
 
 
-def workspace_size(dims: Dims, slots: int, oldest: int, n_valid: int, batch: int, n_sink: int = 0) -> int:
-    """Bytes of the attention workspace (the window's rotated RoPE keys)."""
+def workspace_size(dims: Dims, slots: int, oldest: int, n_valid: int, batch: int, n_sink: int = 0,
+                   n_query: Optional[int] = None) -> int:
+    """Bytes of the attention workspace: the window's rotated RoPE keys, plus the
+    split-KV partials of the preferred split when ``n_query`` is given."""
     cd, win = c_dims(dims), CWindow(slots, oldest, n_valid)
-    return int(load_library().videomla_attention_sink_workspace_size(ctypes.byref(cd), ctypes.byref(win), n_sink,
-                                                                     batch))
+    lib = load_library()
+    if n_query is None:
+        return int(lib.videomla_attention_sink_workspace_size(ctypes.byref(cd), ctypes.byref(win), n_sink, batch))
+    return int(lib.videomla_attention_workspace_size_split(ctypes.byref(cd), ctypes.byref(win), n_sink, batch,
+                                                           n_query))
 
 
 def attention(q_nope: torch.Tensor, q_rope: torch.Tensor, W_uk: torch.Tensor, W_uv: torch.Tensor,
@@ -212,6 +221,8 @@ def attention(q_nope: torch.Tensor, q_rope: torch.Tensor, W_uk: torch.Tensor, W_
     cd = c_dims(dims)
     win = CWindow(slots, oldest, n_valid)
     need = int(lib.videomla_attention_sink_workspace_size(ctypes.byref(cd), ctypes.byref(win), n_sink, B))
+    if workspace is None:  # room for the split-KV partials too
+        need = int(lib.videomla_attention_workspace_size_split(ctypes.byref(cd), ctypes.byref(win), n_sink, B, Nq))
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     elif workspace.device != dev or workspace.numel() * workspace.element_size() < need:

@@ -295,3 +295,39 @@ def test_layer_chain_tiny():
     e = _norm_rel(f64(y.cpu()), ref_y)
     print(f"\nlayer chain tiny: y rel {e:.2e}")
     assert e <= LAYER_NORM_REL
+
+
+# ---------------------------------------------------------------------------
+# split-KV: 1560 queries x 12 heads = 156 units do not fill 148 SMs in whole
+# waves, so the key tiles of each unit are shared by several CTAs
+# ---------------------------------------------------------------------------
+
+def test_attention_split_kv_sink_window_sampled_rows():
+    rows = sample_rows(1560, 48, seed=8)
+    _attention_case(I.WAN, B=1, slots=6, oldest=4, n_valid=6, Nq=1560, seed=1004, rows=rows, n_sink=1)
+
+
+def test_attention_split_kv_matches_unsplit_call():
+    """The same call with a workspace too small for any split partials (one CTA
+    per unit) and with the default one (split): both against the oracle."""
+    dims, slots, oldest, Nq = I.WAN, 21, 7, 1560
+    assert V.workspace_size(dims, slots, oldest, slots, 1, n_query=Nq) > V.workspace_size(dims, slots, oldest, slots, 1)
+    w = I.layer_weights(dims, 1005)
+    q = I.queries(dims, 1, Nq, 1006)
+    cache = I.latent_cache(dims, 1, slots, 1007)
+    wd, qd, cd = _dev(w), _dev(q), cache.to(DEV)
+    small = torch.empty(V.workspace_size(dims, slots, oldest, slots, 1), dtype=torch.uint8, device=DEV)
+    o1, l1 = V.attention(qd["q_nope"], qd["q_rope"], wd["W_uk"], wd["W_uv"], cd, dims, slots, oldest, slots,
+                         want_lse=True, workspace=small)
+    o2, l2 = V.attention(qd["q_nope"], qd["q_rope"], wd["W_uk"], wd["W_uv"], cd, dims, slots, oldest, slots,
+                         want_lse=True)
+    torch.cuda.synchronize()
+    assert V.device_status(reset=True) == V.OK
+    rows = sample_rows(Nq, 32, seed=9)
+    ref_out, ref_lse = oracle_attention(dims, q, w, cache, slots, oldest, slots, rows)
+    for o, l, what in ((o1, l1, "unsplit"), (o2, l2, "split")):
+        got, got_l = f64(o.cpu())[:, rows], f64(l.cpu())[:, rows]
+        check_attention(got, ref_out, f"split-KV {what}")
+        check_lse(got_l, ref_lse, f"split-KV {what} lse")
+    d = np.max(np.abs(f64(o1.cpu()) - f64(o2.cpu())))
+    print(f"\nsplit vs unsplit: max abs diff {d:.2e}")
