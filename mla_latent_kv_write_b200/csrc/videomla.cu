@@ -648,6 +648,6 @@ int videomla_selftest_wait_timeout(uint64_t timeout_ns, void* stream) {
     return cudaGetLastError() == cudaSuccess ? VIDEOMLA_OK : VIDEOMLA_ECUDA;
 }
 
-int videomla_version(void) { return 100; }
+int videomla_version(void) { return 200; }
 
 }  // extern "C"
