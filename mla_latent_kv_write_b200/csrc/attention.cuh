@@ -215,7 +215,9 @@ __global__ void __launch_bounds__(256) rope_window_kernel(const __nv_bfloat16* _
     reinterpret_cast<uint4*>(krot + dst * DR)[ch] = o;
 }
 
-template <class C>
+// SPLIT: this launch shares the key tiles of a unit over p.n_split CTAs (the
+// split-KV epilogue is compiled only into that instance).
+template <class C, bool SPLIT>
 __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant__ AttnMaps maps, const AttnParams p) {
     constexpr int DC = C::DC, DR = C::DR, DN = C::DN, DV = C::DV, BM = C::BM, BK = C::BK, NS = C::NS;
     extern __shared__ uint8_t smem_raw[];
@@ -226,10 +228,12 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
     auto stage = [&](int s) { return smem + s * C::STAGE; };
 
     const int warp = warp_id(), lane = lane_id();
-    const int h = blockIdx.y, b = blockIdx.z / p.n_split, split = blockIdx.z % p.n_split;
+    const int h = blockIdx.y;
+    const int b = SPLIT ? int(blockIdx.z) / p.n_split : int(blockIdx.z);
+    const int split = SPLIT ? int(blockIdx.z) % p.n_split : 0;
     const int q0 = blockIdx.x * BM;
-    const int kt0 = split * p.tiles_per_split;                      // first key tile of this split
-    const int nt = min(p.n_kt, kt0 + p.tiles_per_split) - kt0;     // key tiles of this CTA (>= 1)
+    const int kt0 = SPLIT ? split * p.tiles_per_split : 0;                       // first key tile of this split
+    const int nt = SPLIT ? min(p.n_kt, kt0 + p.tiles_per_split) - kt0 : p.n_kt;  // key tiles of this CTA (>= 1)
     const uint64_t to = p.timeout_ns;
 
     if (threadIdx.x == 0) {
@@ -650,7 +654,7 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
             }
         }
         const int unit = (b * p.H + h) * int(gridDim.x) + int(blockIdx.x);
-        if (ok && p.n_split > 1) {
+        if (SPLIT && ok) {
             // (1) this split's unnormalised O and (max, sum) -> workspace
             const size_t slot = size_t(unit) * p.n_split + split;
             float* po = p.part_o + slot * (BM * DC);
@@ -748,7 +752,7 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                     v[4 * k + 2] = __uint_as_float(o[4 * k + 2]) * f_own[1];
                     v[4 * k + 3] = __uint_as_float(o[4 * k + 3]) * f_own[1];
                 }
-                if (p.n_split > 1) {
+                if constexpr (SPLIT) {
                     for (int sp = 0; sp < p.n_split; ++sp) {
                         if (sp == split) continue;
                         const float* ps = p.part_o + (size_t(unit) * p.n_split + sp) * (BM * DC);

@@ -373,7 +373,7 @@ int run_attention(const videomla_dims* d, const void* q_nope, const void* q_rope
         vmla::rope_window_kernel<DC, DR><<<blocks, 256, 0, st>>>(cache_b, sink_b, static_cast<__half*>(workspace), p, B);
     }
     // 2) latent attention
-    auto kern = vmla::attention_kernel<C>;
+    auto kern = p.n_split > 1 ? vmla::attention_kernel<C, true> : vmla::attention_kernel<C, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
         return VIDEOMLA_ECUDA;
     dim3 grid((Nq + C::BM - 1) / C::BM, H, B * p.n_split);
