@@ -331,3 +331,18 @@ def test_attention_split_kv_matches_unsplit_call():
         check_lse(got_l, ref_lse, f"split-KV {what} lse")
     d = np.max(np.abs(f64(o1.cpu()) - f64(o2.cpu())))
     print(f"\nsplit vs unsplit: max abs diff {d:.2e}")
+
+
+def test_attention_split_kv_batch_two_sampled_rows():
+    """1560 queries x 12 heads x batch 2 = 312 units: split over 4 CTAs, so the
+    grid's z index carries both the batch element and the split."""
+    rows = sample_rows(1560, 24, seed=10)
+    _attention_case(I.WAN, B=2, slots=21, oldest=20, n_valid=21, Nq=1560, seed=1008, rows=rows)
+
+
+def test_attention_split_kv_q_in_shared_memory():
+    """d_c = 384 (Q in shared memory, 64-key tiles, two N = 192 MMA halves) with
+    1560 queries: split-KV merge over the wide latent."""
+    dims = I.sweep_dims(384, 32)
+    rows = sample_rows(1560, 24, seed=11)
+    _attention_case(dims, B=1, slots=21, oldest=3, n_valid=21, Nq=1560, seed=1009, rows=rows)
