@@ -557,7 +557,70 @@ def side_workloads(dev, peak: float):
     torch.cuda.empty_cache()
     res["dense_mha_library"] = dense_mha_library(dev, d, wl.n_query, wl.slots * d.tokens_per_frame)
     res["layer_step"] = layer_step(dev, peak)
+    res["rolling"] = rolling_steps(dev, peak)
+    res["long_window"] = long_window(dev, peak)
     return res
+
+
+def rolling_steps(dev, peak: float):
+    """The 40-step rolling workload: each step writes one frame (1560 tokens)
+    into the 21-slot ring and attends its 1560 queries over the valid window;
+    steps 20-39 (full, wrapping window) are timed back to back."""
+    from mla_latent_kv_write_b200 import videomla as V
+    wl = I.WORKLOADS["rolling"]
+    d = wl.dims
+    T_f = d.tokens_per_frame
+    seed = I.seed_for(wl.index, 0, 0)
+    w = {n: t.to(dev) for n, t in I.layer_weights(d, seed).items()}
+    xs = [I.tokens(d, wl.batch, T_f, seed + 100 + s).to(dev) for s in range(4)]
+    qs = [{n: t.to(dev) for n, t in I.queries(d, wl.batch, T_f, seed + 200 + s).items()} for s in range(4)]
+    cache = torch.zeros(wl.batch, wl.slots * T_f, d.cache_width, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(wl.batch, T_f, d.n_heads, d.d_v, dtype=torch.bfloat16, device=dev)
+
+    def do_step(s):
+        slot = s % wl.slots
+        n_valid = min(s + 1, wl.slots)
+        oldest = 0 if s + 1 <= wl.slots else (slot + 1) % wl.slots
+        V.cache_write(xs[s % 4], w["W_dkv"], w["W_kr"], w["gamma"], cache, d, wl.slots, slot)
+        q = qs[s % 4]
+        V.attention(q["q_nope"], q["q_rope"], w["W_uk"], w["W_uv"], cache, d, wl.slots, oldest, n_valid, out=out)
+
+    for s in range(20):
+        do_step(s)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for s in range(20, wl.steps):
+        do_step(s)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / (wl.steps - 20)
+    fl = flops_cache_write(d, wl.batch, T_f) + flops_attention(d, wl.batch, T_f, wl.slots * T_f)
+    ctas = (T_f + 127) // 128 * d.n_heads * wl.batch
+    return {"workload": "rolling: 1 frame (1560 tokens) per step into a 21-slot ring, steps 20-39 timed",
+            "ms_per_step": ms, "tflops": fl / (ms * 1e-3) / 1e12, "frac": fl / (ms * 1e-3) / 1e12 / peak,
+            "attention_ctas": ctas}
+
+
+def long_window(dev, peak: float):
+    """Minute-scale window: batch 2, 63-frame ring (98,280 keys), 4680 queries."""
+    from mla_latent_kv_write_b200 import videomla as V
+    wl = I.WORKLOADS["long"]
+    d = wl.dims
+    T_f = d.tokens_per_frame
+    calls = []
+    for k in range(2):
+        seed = I.seed_for(wl.index, k, 0)
+        w = {n: t.to(dev) for n, t in I.layer_weights(d, seed).items()}
+        q = {n: t.to(dev) for n, t in I.queries(d, wl.batch, wl.chunk * T_f, seed + 1).items()}
+        cache = I.latent_cache(d, wl.batch, wl.slots, seed + 2).to(dev)
+        out = torch.empty(wl.batch, wl.chunk * T_f, d.n_heads, d.d_v, dtype=torch.bfloat16, device=dev)
+        calls.append(lambda w=w, q=q, cache=cache, out=out: V.attention(
+            q["q_nope"], q["q_rope"], w["W_uk"], w["W_uv"], cache, d, wl.slots, 0, wl.slots, out=out))
+    ms = _time_attention_calls(calls, 3)
+    fl = flops_attention(d, wl.batch, wl.chunk * T_f, wl.slots * T_f)
+    return {"workload": "long: batch 2, 63-frame ring (98280 keys), 4680 queries", "ms": ms,
+            "tflops": fl / (ms * 1e-3) / 1e12, "frac": fl / (ms * 1e-3) / 1e12 / peak}
 
 
 def layer_step(dev, peak: float):
