@@ -36,6 +36,13 @@
 
 namespace vmla {
 
+// max(a, b, c) in one instruction (three-operand form of max.f32, sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 struct AttnParams {
     int Nq, H;
     int T_f, grid_w, slots, oldest;
@@ -545,8 +552,8 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
             for (int c = 0; c < NC; ++c)
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    mx[0] = fmaxf(mx[0], fmaxf(__uint_as_float(sv[c][4 * k]), __uint_as_float(sv[c][4 * k + 1])));
-                    mx[1] = fmaxf(mx[1], fmaxf(__uint_as_float(sv[c][4 * k + 2]), __uint_as_float(sv[c][4 * k + 3])));
+                    mx[0] = fmax3(mx[0], __uint_as_float(sv[c][4 * k]), __uint_as_float(sv[c][4 * k + 1]));
+                    mx[1] = fmax3(mx[1], __uint_as_float(sv[c][4 * k + 2]), __uint_as_float(sv[c][4 * k + 3]));
                 }
 #pragma unroll
             for (int k = 0; k < 2; ++k) {  // the 4 threads of a row hold its 128 columns
@@ -604,23 +611,32 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                 }
             }
             // P = exp2(s * sl - m * sl), packed bf16 pairs for the 16x128b store:
-            // rep kk (4 columns) <- pair (8k + 2 quad, +1) of column half c, kk = 8c + k
-            const float nm0 = -m_used[0] * sl, nm1 = -m_used[1] * sl;
+            // rep kk (4 columns) <- pair (8k + 2 quad, +1) of column half c, kk = 8c + k.
+            // The affine step and the row sums run as paired fp32 ops (one issue
+            // slot per two columns); the softmax warps are issue-bound.
+            const float2 sl2 = make_float2(sl, sl);
+            const float2 nm0 = make_float2(-m_used[0] * sl, -m_used[0] * sl);
+            const float2 nm1 = make_float2(-m_used[1] * sl, -m_used[1] * sl);
+            float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
             uint32_t pa[2 * 8 * NC];
 #pragma unroll
             for (int c = 0; c < NC; ++c)
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const int kk = 8 * c + k;
-                    const float a0 = ex2(fmaf(__uint_as_float(sv[c][4 * k + 0]), sl, nm0));
-                    const float a1 = ex2(fmaf(__uint_as_float(sv[c][4 * k + 1]), sl, nm0));
-                    const float a2 = ex2(fmaf(__uint_as_float(sv[c][4 * k + 2]), sl, nm1));
-                    const float a3 = ex2(fmaf(__uint_as_float(sv[c][4 * k + 3]), sl, nm1));
-                    l_part[0] += a0 + a1;
-                    l_part[1] += a2 + a3;
-                    pa[2 * kk + 0] = pack_bf16(a0, a1);
-                    pa[2 * kk + 1] = pack_bf16(a2, a3);
+                    const float2 x01 = __ffma2_rn(
+                        make_float2(__uint_as_float(sv[c][4 * k + 0]), __uint_as_float(sv[c][4 * k + 1])), sl2, nm0);
+                    const float2 x23 = __ffma2_rn(
+                        make_float2(__uint_as_float(sv[c][4 * k + 2]), __uint_as_float(sv[c][4 * k + 3])), sl2, nm1);
+                    const float2 e01 = make_float2(ex2(x01.x), ex2(x01.y));
+                    const float2 e23 = make_float2(ex2(x23.x), ex2(x23.y));
+                    acc0 = __fadd2_rn(acc0, e01);
+                    acc1 = __fadd2_rn(acc1, e23);
+                    pa[2 * kk + 0] = pack_bf16(e01.x, e01.y);
+                    pa[2 * kk + 1] = pack_bf16(e23.x, e23.y);
                 }
+            l_part[0] += acc0.x + acc0.y;
+            l_part[1] += acc1.x + acc1.y;
             if (j > 0 && !waited) {  // P_{j-1} must have been consumed before P_j overwrites it
                 ok = __all_sync(0xffffffffu, mbar_wait(&bar->pv_done, (j - 1) & 1, ab, to, 43));
                 if (!ok) break;
