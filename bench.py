@@ -98,7 +98,7 @@ def ncu_traffic(kernel: str):
 
 class ClockSampler:
     """SM clock, power and clock-event (throttle) reasons of this rank's GPU while
-    the timed region runs: NVML read every 10 ms from a thread (device found by
+    the timed region runs: NVML read every 2 ms from a thread (device found by
     its PCI bus id, so CUDA_VISIBLE_DEVICES cannot point it at another GPU), or
     nvidia-smi every 200 ms if NVML is unavailable.  Reads only."""
 
@@ -141,10 +141,10 @@ class ClockSampler:
                         self.rows.append((sm, max_sm, pw, rs))
                     except Exception:
                         pass
-                    self.stop.wait(0.01)
+                    self.stop.wait(0.002)
             self.thread = threading.Thread(target=run, daemon=True)
             self.thread.start()
-            self.source = "nvml, 10 ms"
+            self.source = "nvml, 2 ms"
         except Exception:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
@@ -192,7 +192,8 @@ class ClockSampler:
         loaded = [r for r in rows if r[2] > 200.0] or rows
         reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3]) if v.lower() == "active"})
         return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
-                "power_w_max": max(r[2] for r in rows), "samples": len(loaded), "reasons": reasons,
+                "power_w_max": max(r[2] for r in rows), "samples": len(loaded), "samples_all": len(rows),
+                "sm_mhz_range_all": [min(r[0] for r in rows), max(r[0] for r in rows)], "reasons": reasons,
                 "source": self.source}
 
 
