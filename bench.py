@@ -742,6 +742,35 @@ def cache_write_stack(dev, layers: int = 30, reps: int = 3):
             "tflops": flops_cache_write(d, 1, n_tok) / (ms * 1e-3) / 1e12}
 
 
+def profile_sweep(spec: str) -> int:
+    """Three attention calls on one (d_c, d_rope) point of the rank / RoPE sweep
+    (3 query frames vs a 21-frame window, the bench's seeded inputs), nothing
+    timed: a short command for a profiler to capture one launch of that kernel."""
+    from mla_latent_kv_write_b200 import videomla as V
+    d_c, d_rope = (int(v) for v in spec.split(","))
+    if (d_c, d_rope) not in I.SWEEP_POINTS:
+        raise SystemExit(f"--profile-sweep: {spec} is not one of {I.SWEEP_POINTS}")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    V.load_library()
+    wl = WORKLOAD
+    d = I.sweep_dims(d_c, d_rope)
+    seed = I.seed_for(5, 0, wl.slots)
+    w = {n: t.to(dev) for n, t in I.layer_weights(d, seed).items()}
+    q = {n: t.to(dev) for n, t in I.queries(d, 1, wl.n_query, seed + 1).items()}
+    cache = I.latent_cache(d, 1, wl.slots, seed + 2).to(dev)
+    ws = torch.empty(V.workspace_size(d, wl.slots, 0, wl.slots, 1), dtype=torch.uint8, device=dev)
+    out = torch.empty(1, wl.n_query, d.n_heads, d.d_v, dtype=torch.bfloat16, device=dev)
+    for _ in range(3):
+        V.attention(q["q_nope"], q["q_rope"], w["W_uk"], w["W_uv"], cache, d, wl.slots, 0, wl.slots,
+                    out=out, workspace=ws)
+    torch.cuda.synchronize()
+    if V.device_status(reset=True) != V.OK:
+        raise RuntimeError("a kernel reported a timed-out device wait")
+    print(f"profile-sweep {d_c},{d_rope}: 3 attention calls done")
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -750,7 +779,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-side", action="store_true", help="skip the sink-window and sweep side measurements")
+    ap.add_argument("--profile-sweep", metavar="D_C,D_ROPE",
+                    help="only run three attention calls of one rank-sweep point (for a profiler), then exit")
     args = ap.parse_args()
+    if args.profile_sweep:
+        return profile_sweep(args.profile_sweep)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
