@@ -273,8 +273,24 @@ def cpu_oracle_sample(target_s: float = 12.0):
                       f"{d.n_heads} heads, all {wl.slots * T_f} keys; cache write not timed"}
 
 
+def workload_config(world: int) -> dict:
+    """The ``config`` object of the JSON line, the same for both arms."""
+    wl = WORKLOAD
+    d = wl.dims
+    Nk = wl.slots * d.tokens_per_frame
+    return {
+        "workload": "wan_layer: Wan-1.3B-shaped VideoMLA layer, B=1, 12 heads, d_c=192, d_rope=32, "
+                    "d_nope=96, d_v=128, 30x52 grid, cache_write of 3 frames (4680 tokens) into a "
+                    "21-slot ring + attention of 4680 queries x 32760 keys",
+        "global_batch": wl.batch * world, "query_tokens_per_step": wl.n_query, "keys": Nk,
+        "parallelism": f"replicas x{world} (no data-path collective)",
+        "l2": f"inputs larger than L2: {N_SETS} rotating input sets (~60 MB each)",
+        "flops_per_step": flops_attention(d, wl.batch, wl.n_query, Nk) + flops_cache_write(d, wl.batch, wl.n_query),
+    }
+
+
 def run_reference(args):
-    world, rank, _ = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
+    world, rank = int(os.environ.get("WORLD_SIZE", str(args.gpus))), int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     vals = []
@@ -285,13 +301,11 @@ def run_reference(args):
             vals.append(r["value"])
             base = r
     v = statistics.mean(vals)
-    d = WORKLOAD.dims
     line = {
-        "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": base["seconds"] * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"wan_layer: B=1, 12 heads, d_c=192, d_rope=32, 4680 queries x 32760 keys "
-                               f"(oracle on a bounded row sample per step)"},
+        "config": workload_config(world),
         "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": base["cores"], "kind": "oracle",
                          "sample": base["sample"]},
         "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -463,15 +477,7 @@ def run_gpu(args):
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {
-                "workload": "wan_layer: Wan-1.3B-shaped VideoMLA layer, B=1, 12 heads, d_c=192, d_rope=32, "
-                            "d_nope=96, d_v=128, 30x52 grid, cache_write of 3 frames (4680 tokens) into a "
-                            "21-slot ring + attention of 4680 queries x 32760 keys",
-                "global_batch": wl.batch * world, "query_tokens_per_step": wl.n_query, "keys": Nk,
-                "parallelism": f"replicas x{world} (no data-path collective)",
-                "l2": f"inputs larger than L2: {N_SETS} rotating input sets (~60 MB each)",
-                "flops_per_step": fl_step,
-            },
+            "config": workload_config(world),
             "roofline": {"bound": "tensor", "kernel": "attention_kernel", "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak,
                          "peak_kind": f"{peak_src} bf16 {'sustained' if sustained else 'burst'} "

@@ -53,3 +53,14 @@ def test_clock_summary_without_samples():
     c = bench.ClockSampler(0)
     s = c.summary()
     assert s["sm_mhz"] is None and s["reasons"] == ["no samples"]
+
+
+def test_both_arms_share_the_workload_config():
+    # both arms print the same config object, so their lines compare directly
+    c = bench.workload_config(1)
+    assert c["flops_per_step"] == bench.flops_attention(I.WAN, 1, 4680, 32760) + bench.flops_cache_write(I.WAN, 1, 4680)
+    assert c["keys"] == 32760 and c["query_tokens_per_step"] == 4680 and c["global_batch"] == 1
+    assert bench.workload_config(4)["global_batch"] == 4
+    import inspect
+    for fn in (bench.run_reference, bench.run_gpu):
+        assert "workload_config(world)" in inspect.getsource(fn)
