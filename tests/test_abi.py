@@ -154,3 +154,29 @@ def test_attention_sink_rejects_bad_arguments(lib):
     assert call(sink=ctypes.c_void_p(0x10008)) == V.EINVAL         # misaligned sink cache
     assert call(nq=7 * T_f + 1) == V.EINVAL                        # more queries than sink + window tokens
     assert call(ws_bytes=ws - 1) == V.EINVAL                       # workspace without the sink rows
+
+
+def test_split_workspace_follows_the_wave_count(lib):
+    """Split-KV only when the (query tile, head, batch) units leave the last wave of
+    a 148-SM grid mostly empty: the Wan chunk (37 query tiles x 12 heads = 444 units,
+    three full waves) is not split; one query frame (13 x 12 = 156 units, 148 + 8)
+    is, and its workspace adds fp32 partial O tiles and per-row (max, sum) of every
+    split plus one arrival counter per unit.  Without a device the library assumes
+    148 SMs, the B200's count."""
+    d = _dims()
+    T_f = d.grid_h * d.grid_w
+    win = V.CWindow(21, 0, 21)
+    rope = lib.videomla_attention_workspace_size(ctypes.byref(d), ctypes.byref(win), 1)
+    assert rope == 21 * T_f * d.d_rope * 2
+    full = lib.videomla_attention_workspace_size_split(ctypes.byref(d), ctypes.byref(win), 0, 1, 3 * T_f)
+    assert full == rope
+    one = lib.videomla_attention_workspace_size_split(ctypes.byref(d), ctypes.byref(win), 0, 1, T_f)
+    units = 13 * 12
+    per_split = units * (128 * d.d_c * 4 + 128 * 2 * 4)
+    extra = one - (rope + 255) // 256 * 256
+    counters = (units * 4 + 255) // 256 * 256
+    assert (extra - counters) % per_split == 0
+    assert 2 <= (extra - counters) // per_split <= 4
+    # a bad window sizes nothing
+    assert lib.videomla_attention_workspace_size_split(ctypes.byref(d), ctypes.byref(V.CWindow(21, 0, 22)), 0, 1,
+                                                       T_f) == 0
