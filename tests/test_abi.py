@@ -180,3 +180,48 @@ def test_split_workspace_follows_the_wave_count(lib):
     # a bad window sizes nothing
     assert lib.videomla_attention_workspace_size_split(ctypes.byref(d), ctypes.byref(V.CWindow(21, 0, 22)), 0, 1,
                                                        T_f) == 0
+
+
+C_CALLER = r"""
+#include <stdio.h>
+#include <string.h>
+#include "videomla.h"
+
+int main(void) {
+    videomla_dims d;
+    videomla_window w;
+    memset(&d, 0, sizeof d);
+    d.d_model = 1536; d.n_heads = 12; d.d_c = 192; d.d_rope = 32; d.d_nope = 96; d.d_v = 128;
+    d.grid_h = 30; d.grid_w = 52; d.pairs_t = 6; d.pairs_h = 5; d.pairs_w = 5;
+    d.rope_base = 10000.0f; d.rms_eps = 1e-6f;
+    w.slots = 21; w.oldest_slot = 0; w.n_valid = 21;
+    printf("%d|%s|%zu\n", videomla_version(), videomla_strerror(VIDEOMLA_EINVAL),
+           videomla_attention_workspace_size(&d, &w, 1));
+    return 0;
+}
+"""
+
+
+def test_plain_c_caller_links_and_calls_host_entry_points(lib):
+    """The header is C (no C++ in the declarations) and the library exports
+    unmangled names: a C99 program includes it, links the library and calls
+    the entry points that need no device."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    out = os.path.join(ROOT, "_build", "abi_c")
+    os.makedirs(out, exist_ok=True)
+    src = os.path.join(out, "caller.c")
+    with open(src, "w") as f:
+        f.write(C_CALLER)
+    exe = os.path.join(out, "caller")
+    pkg = os.path.dirname(vbuild.LIB)
+    subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"), src,
+                    "-L", pkg, "-lvideomla", "-Wl,-rpath," + pkg, "-o", exe], check=True)
+    r = subprocess.run([exe], check=True, capture_output=True, text=True)
+    version, err, ws = r.stdout.strip().split("|")
+    assert int(version) == lib.videomla_version()
+    assert err == lib.videomla_strerror(V.EINVAL).decode()
+    assert int(ws) == 21 * 1560 * 32 * 2
