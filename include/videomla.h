@@ -96,6 +96,9 @@ typedef struct videomla_window {
  *          slot holds token p of its frame as [RMSNorm(c) | k^R] (k^R unrotated
  *          and unnormalised).  Rows of other slots are untouched.
  *   flags  VIDEOMLA_CACHE_RAW_LATENT to skip the RMSNorm, else 0.
+ * One launch on ``stream``: a chunk of few 128-token tiles (fewer than half the
+ * SMs) spreads each tile's d_model range over a thread-block cluster; more
+ * tiles stream through a persistent kernel (one CTA per SM).  No workspace.
  * Arithmetic: bf16 inputs, fp32 accumulation and normalisation, bf16 RNE output.
  * Errors: EINVAL (null, n_tok not a whole number of frames, first_slot out of
  * range, n_tok / T_f > slots, misaligned), EUNSUPPORTED (d_c + d_rope or d_model
@@ -247,23 +250,32 @@ int videomla_output_projection(const videomla_dims* dims, const void* o, int bat
  * For callers that cannot allocate device memory themselves -- for example a
  * host framework whose memory is owned by a pool or arena it does not expose,
  * code running where cudaMalloc is not allowed or would break a capture, or a
- * plug-in that may only use the buffers it is handed.  The window's rotated
- * RoPE keys go to a fixed scratch array compiled into the library
- * (VIDEOMLA_STATIC_WORKSPACE_BYTES per device, held from library load until
- * process exit).  The function itself allocates nothing and frees nothing.
+ * plug-in that may only use the buffers it is handed.  The call's scratch lives
+ * in a fixed array compiled into the library (VIDEOMLA_STATIC_WORKSPACE_BYTES
+ * per device, held from library load until process exit): the window's rotated
+ * RoPE keys and, when they fit beside them, the split-KV partials and arrival
+ * counters of videomla_attention_workspace_size_split().  The function itself
+ * allocates nothing and frees nothing.
  *
  * Arguments, results and arithmetic are those of videomla_attention.
  * - Sizes: if videomla_attention_workspace_size(dims, window, batch) exceeds
  *   VIDEOMLA_STATIC_WORKSPACE_BYTES the call returns VIDEOMLA_EINVAL and
- *   launches nothing.
- * - Set-up: the first call on each device looks up the device address of the
- *   scratch array with that device current (cudaGetSymbolAddress), which may
- *   load the library's kernels; make that first call before any stream capture.
+ *   launches nothing.  When the preferred split's partials do not fit beside
+ *   the RoPE keys the call runs with the largest split that fits, or unsplit:
+ *   the 1560-query Wan frame step (156 units, 2-4 splits of 31-62 MB) runs
+ *   unsplit here, a few query tiles against a long window (e.g. 128 queries,
+ *   12 heads, 21 Wan frames: 4.8 MB of partials) keep their split.  Results
+ *   agree with videomla_attention to rounding either way.
+ * - Set-up: every call looks up the device address of the scratch array in the
+ *   current context (cudaGetSymbolAddress); the first such lookup on a device
+ *   may load the library's kernels, so make the first call before any stream
+ *   capture.
  * - Sharing: every call on a device uses the same scratch array and leaves the
- *   last call's contents in it.  Nothing in it needs to start at zero (each call
- *   rewrites every row it reads).  Calls whose kernels can overlap on the GPU
- *   (different streams without ordering between them) race on the array; issue
- *   them on one stream or order them.
+ *   last call's contents in it.  Nothing in it needs to start at zero: each call
+ *   rewrites every RoPE row it reads, and the window pre-pass of each call zeroes
+ *   the split counters before the attention kernel uses them.  Calls whose
+ *   kernels can overlap on the GPU (different streams without ordering between
+ *   them) race on the array; issue them on one stream or order them.
  */
 int videomla_attention_static_workspace(const videomla_dims* dims, const void* q_nope, const void* q_rope,
                                         const void* W_uk, const void* W_uv, const void* cache,

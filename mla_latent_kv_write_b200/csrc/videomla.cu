@@ -113,6 +113,15 @@ bool basic_dims_ok(const videomla_dims* d) {
 // ----------------------------------------------------------------------------
 // cache_write
 // ----------------------------------------------------------------------------
+// SM count of the current device (148 on B200).
+int sm_count() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                   cudaSuccess || sms <= 0)
+        return 148;
+    return sms;
+}
+
 // K split of the cache write: CTAs per cluster (1-4) dividing the K chunks.
 // Clusters are placed inside one GPC, so the number that fit at once
 // (cudaOccupancyMaxActiveClusters) decides the waves; pick the split with the
@@ -162,9 +171,9 @@ int pick_ksplit(K kern, int threads, int smem, int chunks, int clusters, int max
 }
 
 template <int DC, int DR>
-int run_cache_write(const videomla_dims* d, const void* x, int B, int n_tok, const void* W_dkv, const void* W_kr,
+int run_cache_write_cluster(const videomla_dims* d, const void* x, int B, int n_tok, const void* W_dkv, const void* W_kr,
                     const float* gamma, void* cache, int slots, int first_slot, unsigned flags, cudaStream_t st) {
-    using C = vmla::CacheWriteCfg<DC, DR>;
+    using C = vmla::ClusterWriteCfg<DC, DR>;
     const int T_f = d->grid_h * d->grid_w;
     CUtensorMap tx, tw, tr;
     {
@@ -185,7 +194,7 @@ int run_cache_write(const videomla_dims* d, const void* x, int B, int n_tok, con
         const uint32_t box[2] = {64, uint32_t(DR)};
         if (!make_map(&tr, W_kr, 2, dims, str, box, 128)) return VIDEOMLA_ECUDA;
     }
-    auto kern = vmla::cache_write_kernel<DC, DR>;
+    auto kern = vmla::cache_write_cluster_kernel<DC, DR>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
         return VIDEOMLA_ECUDA;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess)
@@ -193,6 +202,7 @@ int run_cache_write(const videomla_dims* d, const void* x, int B, int n_tok, con
     const int tiles = (n_tok + C::BM - 1) / C::BM;
     const int ksplit = pick_ksplit(kern, C::THREADS, C::SMEM, d->d_model / C::BKK, tiles * B, C::KS_MAX);
     vmla::CacheWriteParams p;
+    std::memset(&p, 0, sizeof(p));
     p.n_tok = n_tok;
     p.d_model = d->d_model;
     p.ksplit = ksplit;
@@ -218,6 +228,80 @@ int run_cache_write(const videomla_dims* d, const void* x, int B, int n_tok, con
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, kern, tx, tw, tr, p) != cudaSuccess) return VIDEOMLA_ECUDA;
     return launch_status(kern, C::SMEM);
+}
+
+// Many tiles: the persistent stream kernel, one CTA per SM walking the tiles.
+template <int DC, int DR>
+int run_cache_write_stream(const videomla_dims* d, const void* x, int B, int n_tok, const void* W_dkv,
+                           const void* W_kr, const float* gamma, void* cache, int slots, int first_slot,
+                           unsigned flags, cudaStream_t st) {
+    using C = vmla::StreamWriteCfg<DC, DR>;
+    const int T_f = d->grid_h * d->grid_w;
+    CUtensorMap tx, tw, tr;
+    {
+        const uint64_t dims[3] = {uint64_t(d->d_model), uint64_t(n_tok), uint64_t(B)};
+        const uint64_t str[2] = {uint64_t(d->d_model) * 2, uint64_t(n_tok) * d->d_model * 2};
+        const uint32_t box[3] = {64, 128, 1};
+        if (!make_map(&tx, x, 3, dims, str, box, 128)) return VIDEOMLA_ECUDA;
+    }
+    {
+        const uint64_t dims[2] = {uint64_t(d->d_model), uint64_t(DC)};
+        const uint64_t str[1] = {uint64_t(d->d_model) * 2};
+        const uint32_t box[2] = {64, uint32_t(C::WBOX)};
+        if (!make_map(&tw, W_dkv, 2, dims, str, box, 128)) return VIDEOMLA_ECUDA;
+    }
+    {
+        const uint64_t dims[2] = {uint64_t(d->d_model), uint64_t(DR)};
+        const uint64_t str[1] = {uint64_t(d->d_model) * 2};
+        const uint32_t box[2] = {64, uint32_t(DR)};
+        if (!make_map(&tr, W_kr, 2, dims, str, box, 128)) return VIDEOMLA_ECUDA;
+    }
+    auto kern = vmla::cache_write_stream_kernel<DC, DR>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+        return VIDEOMLA_ECUDA;
+    vmla::CacheWriteParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.n_tok = n_tok;
+    p.d_model = d->d_model;
+    p.tiles = (n_tok + C::BM - 1) / C::BM;
+    p.units = p.tiles * B;
+    p.k_chunks = d->d_model / C::BKK;
+    p.T_f = T_f;
+    p.slots = slots;
+    p.first_slot = first_slot;
+    p.normalize = (flags & VIDEOMLA_CACHE_RAW_LATENT) ? 0 : 1;
+    p.eps = d->rms_eps;
+    p.gamma = gamma;
+    p.cache = static_cast<__nv_bfloat16*>(cache);
+    p.timeout_ns = g_timeout_ns.load();
+    const int sms = sm_count();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.units < sms ? p.units : sms, 1, 1);
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // prologue overlaps the previous kernel
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tx, tw, tr, p) != cudaSuccess) {
+        cudaGetLastError();
+        return VIDEOMLA_ECUDA;
+    }
+    return launch_status(kern, 0);
+}
+
+// A chunk of few tiles (fewer than half the SMs) spreads each tile's K range over
+// a cluster; more tiles stream through the persistent kernel, one tile per SM
+// at a time.
+template <int DC, int DR>
+int run_cache_write(const videomla_dims* d, const void* x, int B, int n_tok, const void* W_dkv, const void* W_kr,
+                    const float* gamma, void* cache, int slots, int first_slot, unsigned flags, cudaStream_t st) {
+    const long long units = (long long)B * ((n_tok + 127) / 128);
+    if (2 * units <= sm_count())
+        return run_cache_write_cluster<DC, DR>(d, x, B, n_tok, W_dkv, W_kr, gamma, cache, slots, first_slot, flags, st);
+    return run_cache_write_stream<DC, DR>(d, x, B, n_tok, W_dkv, W_kr, gamma, cache, slots, first_slot, flags, st);
 }
 
 // ----------------------------------------------------------------------------
@@ -581,20 +665,16 @@ static __device__ __align__(256) unsigned char g_static_workspace[VIDEOMLA_STATI
 
 namespace {
 
-// Device address of g_static_workspace on the current device, looked up once
-// per device with that device current.  nullptr if the lookup fails.
+// Device address of g_static_workspace in the current context, or nullptr.  It
+// is looked up on every call (a cheap host query): a cached address could be
+// stale after cudaDeviceReset or under another context on the same device.
 void* static_workspace_address() {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    static std::mutex mu;
-    static void* addr[64] = {};
-    std::lock_guard<std::mutex> lock(mu);
-    if (addr[dev] == nullptr) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess) return nullptr;
-        addr[dev] = p;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess) {
+        cudaGetLastError();  // leave no sticky error for a later launch check
+        return nullptr;
     }
-    return addr[dev];
+    return p;
 }
 
 }  // namespace

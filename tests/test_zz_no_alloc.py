@@ -3,11 +3,12 @@
 Some callers cannot hand the library a scratch buffer: their device memory is
 owned by a pool or arena they do not expose, or they run where a cudaMalloc is
 not allowed.  ``videomla_attention_static_workspace`` serves them with a scratch
-array compiled into the library.  This test calls it through the C ABI twice in
-a row, on two different windows, and checks each result against the regular
-``videomla_attention`` (caller workspace) on the same inputs, with the tolerance
-the other attention tests use.  It also checks that a window too large for the
-built-in array is refused before anything is launched.
+array compiled into the library.  This test calls it through the C ABI three
+times in a row, on different windows (one of them split-KV), and checks each
+result against the regular ``videomla_attention`` (caller workspace) on the same
+inputs, with the tolerance the other attention tests use.  It also checks that
+a window too large for the built-in array is refused before anything is
+launched.
 """
 import ctypes
 
@@ -51,15 +52,24 @@ def _static_call(f, dims, w, q, cache, slots, oldest, n_valid):
     return out, lse
 
 
-def test_static_workspace_matches_regular_entry_point_twice():
+def test_static_workspace_matches_regular_entry_point_in_a_row():
     f = _entry()
     cases = [
-        # Wan-1.3B layer window (2 MiB of scratch), then a wrapped tiny window with
-        # ragged tiles and batch 2: the second call must not see the first's rows
-        (I.WAN, 1, 21, 0, 21, 4680, 31),
-        (I.TINY, 2, 7, 4, 5, 100, 32),
+        # Wan-1.3B layer window (2 MiB of scratch, unsplit), then one query tile
+        # against the same 21-frame window, which splits its key tiles 4 ways
+        # with the partials and counters in the array behind the RoPE keys, on
+        # top of what the first call left there; then a wrapped tiny window with
+        # ragged tiles and batch 2: no call may see another's rows
+        (I.WAN, 1, 21, 0, 21, 4680, 31, False),
+        (I.WAN, 1, 21, 5, 21, 128, 33, True),
+        (I.TINY, 2, 7, 4, 5, 100, 32, None),
     ]
-    for dims, B, slots, oldest, n_valid, Nq, seed in cases:
+    for dims, B, slots, oldest, n_valid, Nq, seed, splits in cases:
+        rope = V.workspace_size(dims, slots, oldest, n_valid, B)
+        preferred = V.workspace_size(dims, slots, oldest, n_valid, B, n_query=Nq)
+        if splits is not None:
+            # the split path runs iff its partials fit in the array beside the RoPE keys
+            assert (rope < preferred <= STATIC_BYTES) == splits
         w, q, cache = _case(dims, B, slots, oldest, n_valid, Nq, seed)
         got, got_lse = _static_call(f, dims, w, q, cache, slots, oldest, n_valid)
         ref, ref_lse = V.attention(q["q_nope"], q["q_rope"], w["W_uk"], w["W_uv"], cache, dims, slots, oldest,
