@@ -478,6 +478,7 @@ def run_gpu(args):
 
     # ---- cache_write on a 30-layer stack (494 MB > L2), for its HBM roofline
     cw_stack = cache_write_stack(dev)
+    cw_batched = cache_write_batched(dev) if world == 1 and not args.no_side else None
     del sets
     side = side_workloads(dev, measured_peaks()[0]["bf16_tflops"]) if world == 1 and not args.no_side else {}
 
@@ -507,6 +508,7 @@ def run_gpu(args):
             "explicit_mha_equivalent_tflops": flops_explicit_equivalent(d, wl.batch, wl.n_query, Nk)
             / (attn_ms * 1e-3) / 1e12,
             "cache_write_stack": cw_stack,
+            "cache_write_batched": cw_batched,
             **side,
             "e2e": {"value": job_throughput(world, fl_step, e2e_ms, args.steps) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
@@ -582,6 +584,7 @@ def side_workloads(dev, peak: float):
     torch.cuda.empty_cache()
     res["dense_mha_library"] = dense_mha_library(dev, d, wl.n_query, wl.slots * d.tokens_per_frame)
     res["layer_step"] = layer_step(dev, peak)
+    res["projection_ab"] = projection_ab(dev)
     res["rolling"] = rolling_steps(dev, peak)
     res["long_window"] = long_window(dev, peak)
     return res
@@ -683,6 +686,65 @@ def layer_step(dev, peak: float):
             "frac": fl / (ms * 1e-3) / 1e12 / peak, "flops": fl, "projection_flops": fl_q + fl_o}
 
 
+def projection_ab(dev):
+    """The two re-associations the pages give for inference, each timed against
+    the order this library uses (Wan chunk, 4680 tokens, 12 heads, d_c 192):
+      output side (App. E Eq. 10-11): y = sum_h B_h o_lat,h with B_h = W_O,h W_uv,h
+        [d_model x d_c] -- one GEMM with K = H d_c = 2304 on the per-head O_lat / l
+        -- against the attention's W_uv epilogue + y = W_O [o_1 .. o_H] (K = H d_v
+        = 1536);
+      query side (Eq. 9): q_abs,h = A_h^T c^Q with A_h = W_uq,h^T W_uk,h
+        [d_q x d_c] -- the up-projection GEMM widens from H d_nope = 1152 to
+        H d_c = 2304 columns -- against q^nope = W_uq c^Q + the attention's
+        in-kernel absorption.
+    Each GEMM runs through the public entry points (the output projection with
+    d_v := d_c, the query path with d_nope := d_c) on random weights of those
+    shapes, 10 calls per CUDA graph.  The attention-side terms (W_uv epilogue,
+    absorption) are counted in flops: each is under 0.2 % of the attention."""
+    import dataclasses
+    from mla_latent_kv_write_b200 import videomla as V
+    wl, d = WORKLOAD, WORKLOAD.dims
+    M = wl.n_query
+    g = torch.Generator().manual_seed(7100)
+
+    def rnd(*shape, std=1.0):
+        return (torch.randn(*shape, generator=g) * std).to(torch.bfloat16).to(dev)
+    out = {}
+    # output side
+    o = rnd(1, M, d.n_heads, d.d_v)
+    W_O = rnd(d.d_model, d.n_heads * d.d_v, std=(d.n_heads * d.d_v) ** -0.5)
+    y = torch.empty(1, M, d.d_model, dtype=torch.bfloat16, device=dev)
+    d_b = dataclasses.replace(d, d_v=d.d_c)
+    o_lat = rnd(1, M, d.n_heads, d.d_c)
+    B = rnd(d.d_model, d.n_heads * d.d_c, std=(d.n_heads * d.d_c) ** -0.5)
+    t_wo = _graph_time_ms(lambda: [V.output_projection(o, W_O, d, y=y) for _ in range(10)], 5) / 10
+    t_b = _graph_time_ms(lambda: [V.output_projection(o_lat, B, d_b, y=y) for _ in range(10)], 5) / 10
+    fl_wo = 2.0 * M * d.n_heads * d.d_v * d.d_model
+    fl_uv = 2.0 * M * d.n_heads * d.d_c * d.d_v
+    fl_b = 2.0 * M * d.n_heads * d.d_c * d.d_model
+    out["output_side"] = {"built_W_O_gemm_ms": t_wo, "built_gflop": (fl_wo + fl_uv) / 1e9,
+                          "B_h_gemm_ms": t_b, "B_h_gflop": fl_b / 1e9, "faster": "built" if t_wo <= t_b else "B_h"}
+    # query side
+    pw = {n: t.to(dev) for n, t in I.projection_weights(d, 7101).items()}
+    x = rnd(1, M, d.d_model)
+    d_a = dataclasses.replace(d, d_nope=d.d_c)
+    A_t = rnd(d.n_heads * d.d_c, d.d_q, std=d.d_q ** -0.5)
+    qn = torch.empty(1, M, d.n_heads, d.d_nope, dtype=torch.bfloat16, device=dev)
+    qa = torch.empty(1, M, d.n_heads, d.d_c, dtype=torch.bfloat16, device=dev)
+    qr = torch.empty(1, M, d.n_heads, d.d_rope, dtype=torch.bfloat16, device=dev)
+    t_q = _graph_time_ms(lambda: [V.query_projection(x, pw["W_dq"], pw["gamma_q"], pw["W_uq"], pw["W_qr"], d,
+                                                     q_nope=qn, q_rope=qr) for _ in range(10)], 5) / 10
+    t_a = _graph_time_ms(lambda: [V.query_projection(x, pw["W_dq"], pw["gamma_q"], A_t, pw["W_qr"], d_a,
+                                                     q_nope=qa, q_rope=qr) for _ in range(10)], 5) / 10
+    fl_dq = 2.0 * M * d.d_model * d.d_q
+    fl_q = fl_dq + 2.0 * M * d.d_q * d.n_heads * (d.d_nope + d.d_rope)
+    fl_abs = 2.0 * M * d.n_heads * d.d_nope * d.d_c
+    fl_a = fl_dq + 2.0 * M * d.d_q * d.n_heads * (d.d_c + d.d_rope)
+    out["query_side"] = {"built_query_path_ms": t_q, "built_gflop": (fl_q + fl_abs) / 1e9,
+                         "A_h_query_path_ms": t_a, "A_h_gflop": fl_a / 1e9, "faster": "built" if t_q <= t_a else "A_h"}
+    return out
+
+
 def dense_mha_library(dev, d, Nq: int, Nk: int):
     """Same-shape dense multi-head attention through torch's scaled-dot-product
     attention (a library kernel, not this repository's): per-head K and V of
@@ -717,27 +779,13 @@ def dense_mha_library(dev, d, Nq: int, Nk: int):
             "latent_cache_bytes_per_token_layer": 2 * (d.d_c + d.d_rope)}
 
 
-def cache_write_stack(dev, layers: int = 30, reps: int = 3):
-    """cache_write over 30 independent layers (3-frame chunks, 494 MB of x +
-    cache traffic > L2), timed back to back; HBM roofline of that kernel."""
-    from mla_latent_kv_write_b200 import videomla as V
-    wl, d = WORKLOAD, WORKLOAD.dims
-    T_f = d.tokens_per_frame
-    n_tok = wl.chunk * T_f
-    xs, caches, ws = [], [], []
-    for l in range(layers):
-        seed = I.seed_for(4, l, 0)
-        xs.append(I.tokens(d, 1, n_tok, seed).to(dev))
-        ws.append({k: v.to(dev) for k, v in I.layer_weights(d, seed).items()})
-        caches.append(torch.zeros(1, wl.slots * T_f, d.cache_width, dtype=torch.bfloat16, device=dev))
-    def run():
-        for l in range(layers):
-            V.cache_write(xs[l], ws[l]["W_dkv"], ws[l]["W_kr"], ws[l]["gamma"], caches[l], d, wl.slots, wl.prefill)
+def _graph_time_ms(run, reps: int) -> float:
+    """Best-of-``reps`` CUDA-event time of one replay of the calls ``run`` makes,
+    captured into a CUDA graph so that the events time the GPU, not the Python
+    launch loop (a 4680-token cache write takes microseconds, less than the host
+    needs to prepare a call)."""
     run()
     torch.cuda.synchronize()
-    # A 4680-token layer takes a few microseconds on the GPU, less than the host
-    # needs to prepare a call: replay the 30 calls from a CUDA graph so that the
-    # events time the GPU, not the Python launch loop.
     graph = torch.cuda.CUDAGraph()
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
@@ -756,14 +804,69 @@ def cache_write_stack(dev, layers: int = 30, reps: int = 3):
         evs.append((a, b))
     torch.cuda.synchronize()
     del graph
-    ms = min(a.elapsed_time(b) for a, b in evs) / layers
+    return min(a.elapsed_time(b) for a, b in evs)
+
+
+def cache_write_stack(dev, layers: int = 30, reps: int = 3):
+    """cache_write over 30 independent layers (3-frame chunks, 494 MB of x +
+    cache traffic > L2), timed back to back; HBM roofline of that kernel."""
+    from mla_latent_kv_write_b200 import videomla as V
+    wl, d = WORKLOAD, WORKLOAD.dims
+    T_f = d.tokens_per_frame
+    n_tok = wl.chunk * T_f
+    xs, caches, ws = [], [], []
+    for l in range(layers):
+        seed = I.seed_for(4, l, 0)
+        xs.append(I.tokens(d, 1, n_tok, seed).to(dev))
+        ws.append({k: v.to(dev) for k, v in I.layer_weights(d, seed).items()})
+        caches.append(torch.zeros(1, wl.slots * T_f, d.cache_width, dtype=torch.bfloat16, device=dev))
+
+    def run():
+        for l in range(layers):
+            V.cache_write(xs[l], ws[l]["W_dkv"], ws[l]["W_kr"], ws[l]["gamma"], caches[l], d, wl.slots, wl.prefill)
+    ms = _graph_time_ms(run, reps) / layers
     by = bytes_cache_write(d, 1, n_tok)
     gbs = by / (ms * 1e-3) / 1e9
     peaks, src = measured_peaks()
     return {"layers": layers, "timing": "30 calls replayed from one CUDA graph, best of 3",
             "ms_per_layer": ms, "bytes_per_layer": by, "achieved_gbs": gbs,
             "peak_gbs": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"], "peak_kind": f"{src} HBM copy",
-            "tflops": flops_cache_write(d, 1, n_tok) / (ms * 1e-3) / 1e12}
+            "tflops": flops_cache_write(d, 1, n_tok) / (ms * 1e-3) / 1e12,
+            "roofline": {"bound": "hbm", "kernel": "cache_write_cluster_kernel", "achieved": gbs,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                         "peak_kind": f"{src} HBM copy", "algorithmic_bytes_per_launch": by,
+                         "traffic": ncu_traffic("cache_write_cluster_kernel")}}
+
+
+def cache_write_batched(dev, batches=(1, 2, 4, 8), reps: int = 5):
+    """The cache write of a 3-frame chunk for batch 1, 2, 4 and 8 requests in one
+    call: three rotating input sets (x and ring differ per call, > L2 at batch
+    >= 4), six calls per CUDA graph.  With more 128-token tiles than half the SMs
+    the call runs the persistent stream kernel."""
+    from mla_latent_kv_write_b200 import videomla as V
+    wl, d = WORKLOAD, WORKLOAD.dims
+    T_f = d.tokens_per_frame
+    n_tok = wl.chunk * T_f
+    peaks, src = measured_peaks()
+    out = []
+    for B in batches:
+        xs = [I.tokens(d, B, n_tok, I.seed_for(4, 0, 50 + k)).to(dev) for k in range(3)]
+        w = {k: v.to(dev) for k, v in I.layer_weights(d, I.seed_for(4, 0, 60)).items()}
+        caches = [torch.zeros(B, wl.slots * T_f, d.cache_width, dtype=torch.bfloat16, device=dev) for _ in range(3)]
+
+        def run():
+            for k in range(6):
+                V.cache_write(xs[k % 3], w["W_dkv"], w["W_kr"], w["gamma"], caches[k % 3], d, wl.slots,
+                              wl.prefill)
+        ms = _graph_time_ms(run, reps) / 6
+        by = bytes_cache_write(d, B, n_tok)
+        tiles = B * ((n_tok + 127) // 128)
+        out.append({"batch": B, "tiles": tiles,
+                    "kernel": "cache_write_cluster_kernel" if 2 * tiles <= 148 else "cache_write_stream_kernel",
+                    "us_per_call": ms * 1e3, "achieved_gbs": by / (ms * 1e-3) / 1e9,
+                    "frac": by / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]})
+        del xs, caches
+    return out
 
 
 def profile_sweep(spec: str) -> int:

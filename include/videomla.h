@@ -214,7 +214,8 @@ size_t videomla_query_projection_workspace_size(const videomla_dims* dims, int d
  *   W_uq    [n_heads * d_nope, d_q] bf16, W_qr [n_heads * d_rope, d_q] bf16
  *   q_nope  [batch, n_tok, n_heads, d_nope] bf16, q_rope [batch, n_tok, n_heads, d_rope] bf16
  *   workspace  at least videomla_query_projection_workspace_size() bytes, 16-byte aligned.
- * Three tcgen05 GEMM launches and one row-normalisation launch on ``stream``.
+ * Two persistent tcgen05 GEMM launches (the second writes both up-projections)
+ * and one row-normalisation launch on ``stream``.
  * Errors: EINVAL (null, d_q or d_model not a multiple of 64, n_heads * d_nope or
  * n_heads * d_rope not a multiple of 8, small workspace, misaligned), ECUDA.
  */

@@ -467,46 +467,79 @@ int run_attention(const videomla_dims* d, const void* q_nope, const void* q_rope
 
 
 // ----------------------------------------------------------------------------
-// projections: C [M, N] = A [M, K] . B [N, K]^T
+// projections: C_g [M, N_g] = A [M, K] . B_g [N_g, K]^T, one or two column groups
 // ----------------------------------------------------------------------------
 template <int BN, bool F32OUT>
-int run_gemm(const void* A, const void* B, int M, int N, int K, void* Cmat, int ldc, cudaStream_t st) {
+int run_gemm(const void* A, int M, int K, int groups, const void* B0, int N0, void* C0, int ldc0, const void* B1,
+             int N1, void* C1, int ldc1, cudaStream_t st) {
     using C = vmla::GemmCfg<BN, F32OUT>;
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb[2];
     {
         const uint64_t dims[2] = {uint64_t(K), uint64_t(M)};
         const uint64_t str[1] = {uint64_t(K) * 2};
         const uint32_t box[2] = {64, uint32_t(C::BM)};
         if (!make_map(&ta, A, 2, dims, str, box, 128)) return VIDEOMLA_ECUDA;
     }
-    {
-        const uint64_t dims[2] = {uint64_t(K), uint64_t(N)};
+    const void* Bs[2] = {B0, groups > 1 ? B1 : B0};
+    const int Ns[2] = {N0, groups > 1 ? N1 : N0};
+    for (int g = 0; g < 2; ++g) {
+        const uint64_t dims[2] = {uint64_t(K), uint64_t(Ns[g])};
         const uint64_t str[1] = {uint64_t(K) * 2};
         const uint32_t box[2] = {64, uint32_t(BN)};
-        if (!make_map(&tb, B, 2, dims, str, box, 128)) return VIDEOMLA_ECUDA;
+        if (!make_map(&tb[g], Bs[g], 2, dims, str, box, 128)) return VIDEOMLA_ECUDA;
     }
     auto kern = vmla::gemm_kernel<C>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
         return VIDEOMLA_ECUDA;
     vmla::GemmParams p;
+    std::memset(&p, 0, sizeof(p));
     p.M = M;
-    p.N = N;
     p.K = K;
-    p.C = Cmat;
-    p.ldc = ldc;
+    p.n_groups = groups;
+    p.N[0] = N0;
+    p.N[1] = groups > 1 ? N1 : 0;
+    p.n_tiles[0] = (N0 + BN - 1) / BN;
+    p.n_tiles[1] = groups > 1 ? (N1 + BN - 1) / BN : 0;
+    p.m_tiles = (M + C::BM - 1) / C::BM;
+    p.tiles = p.m_tiles * (p.n_tiles[0] + p.n_tiles[1]);
+    p.C[0] = C0;
+    p.C[1] = C1;
+    p.ldc[0] = ldc0;
+    p.ldc[1] = ldc1;
     p.timeout_ns = g_timeout_ns.load();
-    dim3 grid((M + C::BM - 1) / C::BM, (N + BN - 1) / BN);
-    kern<<<grid, C::THREADS, C::SMEM, st>>>(ta, tb, p);
+    const int sms = sm_count();
+    kern<<<p.tiles < sms ? p.tiles : sms, C::THREADS, C::SMEM, st>>>(ta, tb[0], tb[1], p);
     return launch_status(kern, C::SMEM);
 }
 
-// bf16 C unless f32out; 256-column tiles when they divide N, else 128.
-int gemm(const void* A, const void* B, int M, int N, int K, void* Cmat, int ldc, bool f32out, cudaStream_t st) {
-    if (N % 256 == 0)
-        return f32out ? run_gemm<256, true>(A, B, M, N, K, Cmat, ldc, st) : run_gemm<256, false>(A, B, M, N, K, Cmat, ldc, st);
-    return f32out ? run_gemm<128, true>(A, B, M, N, K, Cmat, ldc, st) : run_gemm<128, false>(A, B, M, N, K, Cmat, ldc, st);
+// Column tile width: the one that puts the fewest columns on the busiest SM of
+// the persistent grid (ties go to 256, fewer tiles).
+int gemm_bn(int M, int N0, int N1, int groups) {
+    const long long m_tiles = (M + 127) / 128;
+    const int sms = sm_count();
+    long long cost[2];
+    const int bns[2] = {256, 128};
+    for (int i = 0; i < 2; ++i) {
+        const int bn = bns[i];
+        const long long t = m_tiles * ((N0 + bn - 1) / bn + (groups > 1 ? (N1 + bn - 1) / bn : 0));
+        cost[i] = (t + sms - 1) / sms * bn;
+    }
+    return cost[1] < cost[0] ? 128 : 256;
 }
 
+// bf16 or fp32 C; one or two column groups sharing A.
+int gemm2(const void* A, int M, int K, int groups, const void* B0, int N0, void* C0, int ldc0, const void* B1, int N1,
+          void* C1, int ldc1, bool f32out, cudaStream_t st) {
+    if (gemm_bn(M, N0, N1, groups) == 256)
+        return f32out ? run_gemm<256, true>(A, M, K, groups, B0, N0, C0, ldc0, B1, N1, C1, ldc1, st)
+                      : run_gemm<256, false>(A, M, K, groups, B0, N0, C0, ldc0, B1, N1, C1, ldc1, st);
+    return f32out ? run_gemm<128, true>(A, M, K, groups, B0, N0, C0, ldc0, B1, N1, C1, ldc1, st)
+                  : run_gemm<128, false>(A, M, K, groups, B0, N0, C0, ldc0, B1, N1, C1, ldc1, st);
+}
+
+int gemm(const void* A, const void* B, int M, int N, int K, void* Cmat, int ldc, bool f32out, cudaStream_t st) {
+    return gemm2(A, M, K, 1, B, N, Cmat, ldc, nullptr, 0, nullptr, 0, f32out, st);
+}
 
 }  // namespace
 
@@ -639,8 +672,8 @@ int videomla_query_projection(const videomla_dims* dims, int d_q, const void* x,
     if (int rc = gemm(x, W_dq, int(M), d_q, dims->d_model, cq, d_q, true, st)) return rc;
     vmla::rms_norm_rows_kernel<<<int((M + 7) / 8), 256, 0, st>>>(cq, cqn, gamma_q, int(M), d_q, dims->rms_eps);
     if (cudaGetLastError() != cudaSuccess) return VIDEOMLA_ECUDA;
-    if (int rc = gemm(cqn, W_uq, int(M), int(nq), d_q, q_nope, int(nq), false, st)) return rc;
-    return gemm(cqn, W_qr, int(M), int(nr), d_q, q_rope, int(nr), false, st);
+    // both up-projections read the normalised c^Q: one launch, two column groups
+    return gemm2(cqn, int(M), d_q, 2, W_uq, int(nq), q_nope, int(nq), W_qr, int(nr), q_rope, int(nr), false, st);
 }
 
 int videomla_output_projection(const videomla_dims* dims, const void* o, int batch, int n_query, const void* W_O,
