@@ -114,6 +114,42 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, AbortS
     return mbar_wait_slow(bar, parity, ab, timeout_ns, site);
 }
 
+// Bounded wait with cluster-scope acquire: for barriers that CTAs of the
+// cluster (or the pair's bulk copies and MMAs) arrive on.
+__device__ __forceinline__ bool mbar_try_wait_cl(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __noinline__ bool mbar_wait_cl_slow(uint64_t* bar, uint32_t parity, AbortState* ab, uint64_t timeout_ns,
+                                               int site) {
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait_cl(bar, parity)) return true;
+        if ((i & 15u) == 0u) {
+            __nanosleep(64);
+            if (ab->flag) return false;
+            if (globaltimer_ns() - t0 > timeout_ns) {
+                ab->flag = 1;
+                atomicCAS(&g_status, 0, -4 - (site << 8));
+                __threadfence();
+                return false;
+            }
+        }
+    }
+}
+__device__ __forceinline__ bool mbar_wait_cl(uint64_t* bar, uint32_t parity, AbortState* ab, uint64_t timeout_ns,
+                                             int site) {
+    if (mbar_try_wait_cl(bar, parity)) return true;
+    return mbar_wait_cl_slow(bar, parity, ab, timeout_ns, site);
+}
+
 // Bounded wait used on the unwind path: ignores the abort flag, so that a role
 // can let its own asynchronous copies / MMAs finish before the CTA releases its
 // tensor memory and exits.  Returns false if even this wait ran out.
@@ -214,6 +250,55 @@ __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// ---- CTA pairs (cta_group::2): one MMA spans the tensor cores of two SMs.
+// The pair is a cluster of 2; rank 0 issues the MMAs.  A's rows split across
+// the pair (each CTA's shared memory holds its 128 rows), B's N columns split
+// across the pair; each CTA's tensor memory holds its 128 rows of D.  Both CTAs
+// allocate the same columns.
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// D (+)= A * B for the pair, both operands from shared memory (same offsets in both CTAs).
+__device__ __forceinline__ void umma_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Completion of the pair's MMAs -> one arrive on the mbarrier at this offset in
+// every CTA of ``cta_mask`` (bit r = cluster rank r).
+__device__ __forceinline__ void umma_commit_pair_mc(uint64_t* bar, uint16_t cta_mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(cta_mask)
+        : "memory");
+}
+// 2D tile load into this CTA's shared memory whose completion is counted on
+// the mbarrier at cluster address ``bar_cluster`` (either CTA of the pair).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m, uint32_t bar_cluster, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+        "%4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(x), "r"(y)
+        : "memory");
+}
+// Arrive on an mbarrier of another CTA of the cluster (cluster address).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
 
 // D (tmem, fp32) (+)= A (tmem, packed bf16) * B (smem desc), kind::f16.

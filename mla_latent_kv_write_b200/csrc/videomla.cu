@@ -469,10 +469,42 @@ int run_attention(const videomla_dims* d, const void* q_nope, const void* q_rope
 // ----------------------------------------------------------------------------
 // projections: C_g [M, N_g] = A [M, K] . B_g [N_g, K]^T, one or two column groups
 // ----------------------------------------------------------------------------
+// Largest number of 2-CTA clusters of a kernel that can be resident at once (cached per device).
+int max_pair_clusters(const void* kern, int threads, int smem) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static std::mutex mu;
+    static int cache[64][2] = {};
+    const int slot = smem > 140000 ? 1 : 0;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (dev >= 0 && dev < 64 && cache[dev][slot] > 0) return cache[dev][slot];
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = sm_count() / 2;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev >= 0 && dev < 64) cache[dev][slot] = n;
+    return n;
+}
+
 template <int BN, bool F32OUT>
-int run_gemm(const void* A, int M, int K, int groups, const void* B0, int N0, void* C0, int ldc0, const void* B1,
-             int N1, void* C1, int ldc1, cudaStream_t st) {
-    using C = vmla::GemmCfg<BN, F32OUT>;
+int run_gemm_pair(const void* A, int M, int K, int groups, const void* B0, int N0, void* C0, int ldc0, const void* B1,
+                  int N1, void* C1, int ldc1, cudaStream_t st) {
+    using C = vmla::GemmPairCfg<BN, F32OUT>;
     CUtensorMap ta, tb[2];
     {
         const uint64_t dims[2] = {uint64_t(K), uint64_t(M)};
@@ -485,10 +517,10 @@ int run_gemm(const void* A, int M, int K, int groups, const void* B0, int N0, vo
     for (int g = 0; g < 2; ++g) {
         const uint64_t dims[2] = {uint64_t(K), uint64_t(Ns[g])};
         const uint64_t str[1] = {uint64_t(K) * 2};
-        const uint32_t box[2] = {64, uint32_t(BN)};
+        const uint32_t box[2] = {64, uint32_t(C::BNH)};
         if (!make_map(&tb[g], Bs[g], 2, dims, str, box, 128)) return VIDEOMLA_ECUDA;
     }
-    auto kern = vmla::gemm_kernel<C>;
+    auto kern = vmla::gemm_pair_kernel<C>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
         return VIDEOMLA_ECUDA;
     vmla::GemmParams p;
@@ -500,41 +532,57 @@ int run_gemm(const void* A, int M, int K, int groups, const void* B0, int N0, vo
     p.N[1] = groups > 1 ? N1 : 0;
     p.n_tiles[0] = (N0 + BN - 1) / BN;
     p.n_tiles[1] = groups > 1 ? (N1 + BN - 1) / BN : 0;
-    p.m_tiles = (M + C::BM - 1) / C::BM;
+    p.m_tiles = (M + 255) / 256;
     p.tiles = p.m_tiles * (p.n_tiles[0] + p.n_tiles[1]);
     p.C[0] = C0;
     p.C[1] = C1;
     p.ldc[0] = ldc0;
     p.ldc[1] = ldc1;
     p.timeout_ns = g_timeout_ns.load();
-    const int sms = sm_count();
-    kern<<<p.tiles < sms ? p.tiles : sms, C::THREADS, C::SMEM, st>>>(ta, tb[0], tb[1], p);
+    const int pairs_max = max_pair_clusters(reinterpret_cast<const void*>(kern), C::THREADS, C::SMEM);
+    const int pairs = p.tiles < pairs_max ? p.tiles : pairs_max;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb[0], tb[1], p) != cudaSuccess) {
+        cudaGetLastError();
+        return VIDEOMLA_ECUDA;
+    }
     return launch_status(kern, C::SMEM);
 }
 
-// Column tile width: the one that puts the fewest columns on the busiest SM of
-// the persistent grid (ties go to 256, fewer tiles).
-int gemm_bn(int M, int N0, int N1, int groups) {
-    const long long m_tiles = (M + 127) / 128;
-    const int sms = sm_count();
+// Column tile width of the pair tiles: the one that puts the fewest columns on
+// the busiest pair of the persistent grid (ties go to 256, fewer tiles).
+int gemm_pair_bn(int M, int N0, int N1, int groups) {
+    const long long m_tiles = (M + 255) / 256;
+    const int pairs = sm_count() / 2;
     long long cost[2];
     const int bns[2] = {256, 128};
     for (int i = 0; i < 2; ++i) {
         const int bn = bns[i];
         const long long t = m_tiles * ((N0 + bn - 1) / bn + (groups > 1 ? (N1 + bn - 1) / bn : 0));
-        cost[i] = (t + sms - 1) / sms * bn;
+        cost[i] = (t + pairs - 1) / pairs * bn;
     }
     return cost[1] < cost[0] ? 128 : 256;
 }
 
-// bf16 or fp32 C; one or two column groups sharing A.
+// bf16 or fp32 C; one or two column groups sharing A; CTA-pair kernel.
 int gemm2(const void* A, int M, int K, int groups, const void* B0, int N0, void* C0, int ldc0, const void* B1, int N1,
           void* C1, int ldc1, bool f32out, cudaStream_t st) {
-    if (gemm_bn(M, N0, N1, groups) == 256)
-        return f32out ? run_gemm<256, true>(A, M, K, groups, B0, N0, C0, ldc0, B1, N1, C1, ldc1, st)
-                      : run_gemm<256, false>(A, M, K, groups, B0, N0, C0, ldc0, B1, N1, C1, ldc1, st);
-    return f32out ? run_gemm<128, true>(A, M, K, groups, B0, N0, C0, ldc0, B1, N1, C1, ldc1, st)
-                  : run_gemm<128, false>(A, M, K, groups, B0, N0, C0, ldc0, B1, N1, C1, ldc1, st);
+    if (gemm_pair_bn(M, N0, N1, groups) == 256)
+        return f32out ? run_gemm_pair<256, true>(A, M, K, groups, B0, N0, C0, ldc0, B1, N1, C1, ldc1, st)
+                      : run_gemm_pair<256, false>(A, M, K, groups, B0, N0, C0, ldc0, B1, N1, C1, ldc1, st);
+    return f32out ? run_gemm_pair<128, true>(A, M, K, groups, B0, N0, C0, ldc0, B1, N1, C1, ldc1, st)
+                  : run_gemm_pair<128, false>(A, M, K, groups, B0, N0, C0, ldc0, B1, N1, C1, ldc1, st);
 }
 
 int gemm(const void* A, const void* B, int M, int N, int K, void* Cmat, int ldc, bool f32out, cudaStream_t st) {
