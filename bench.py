@@ -582,7 +582,8 @@ def side_workloads(dev, peak: float):
         del calls
     res["sweep_attention"] = sweep
     torch.cuda.empty_cache()
-    res["dense_mha_library"] = dense_mha_library(dev, d, wl.n_query, wl.slots * d.tokens_per_frame)
+    lat = next((x["ms"] for x in sweep if (x["d_c"], x["d_rope"]) == (d.d_c, d.d_rope)), None)
+    res["dense_mha"] = dense_mha(dev, d, wl.n_query, wl.slots * d.tokens_per_frame, latent_ms=lat)
     res["layer_step"] = layer_step(dev, peak)
     res["projection_ab"] = projection_ab(dev)
     res["rolling"] = rolling_steps(dev, peak)
@@ -745,21 +746,29 @@ def projection_ab(dev):
     return out
 
 
-def dense_mha_library(dev, d, Nq: int, Nk: int):
-    """Same-shape dense multi-head attention through torch's scaled-dot-product
-    attention (a library kernel, not this repository's): per-head K and V of
-    d_nope + d_rope = 128 channels for every key, the 2 n_h d_h = 3072-scalar
-    cache of the pages' dense baseline ([VideoMLA] App. C.1).  For the same-box
-    time and cache-bytes ratios only; its flops are 4 d_h per (q, k, h)."""
+def dense_mha(dev, d, Nq: int, Nk: int, latent_ms: float):
+    """The pages' dense baseline on the same shape ([VideoMLA] App. C.1): per-head
+    K and V of 128 channels for every key, the 2 n_h d_h = 3072-scalar cache, through
+    this library's dense kernel (``videomla_dense_attention``, parity-tested against
+    the oracle's explicit form), and through torch's scaled-dot-product attention
+    (cuDNN / flash) for reference.  Random K / V of that shape (2 sets of 2 x
+    201 MB, larger than L2); flops 4 d_h per (q, k, h).  The latent call's time is
+    passed in for the ratio."""
     import torch.nn.functional as F
+    from mla_latent_kv_write_b200 import videomla as V
     dh = d.d_nope + d.d_rope
     g = torch.Generator(device="cpu").manual_seed(77)
     sets = []
-    for _ in range(2):   # 2 x 2 x 201 MB of K / V: larger than L2
-        q = torch.randn(1, d.n_heads, Nq, dh, generator=g).to(torch.bfloat16).to(dev)
-        k = torch.randn(1, d.n_heads, Nk, dh, generator=g).to(torch.bfloat16).to(dev)
-        v = torch.randn(1, d.n_heads, Nk, dh, generator=g).to(torch.bfloat16).to(dev)
-        sets.append((q, k, v))
+    for _ in range(2):
+        qn = torch.randn(1, Nq, d.n_heads, d.d_nope, generator=g).to(torch.bfloat16).to(dev)
+        qr = torch.randn(1, Nq, d.n_heads, d.d_rope, generator=g).to(torch.bfloat16).to(dev)
+        k = torch.randn(1, Nk, d.n_heads, dh, generator=g).to(torch.bfloat16).to(dev)
+        v = torch.randn(1, Nk, d.n_heads, dh, generator=g).to(torch.bfloat16).to(dev)
+        o = torch.empty(1, Nq, d.n_heads, dh, dtype=torch.bfloat16, device=dev)
+        sets.append((qn, qr, k, v, o))
+    calls = [lambda qn=qn, qr=qr, k=k, v=v, o=o: V.dense_attention(qn, qr, k, v, d, out=o)
+             for qn, qr, k, v, o in sets]
+    ms_ours = _time_attention_calls(calls, 5)
     backend = "default"
     try:
         from torch.nn.attention import SDPBackend, sdpa_kernel
@@ -768,15 +777,22 @@ def dense_mha_library(dev, d, Nq: int, Nk: int):
     except Exception:  # older torch: its own choice
         import contextlib
         ctx = contextlib.nullcontext()
+    lib_sets = [(torch.cat([qn, qr], -1).transpose(1, 2).contiguous(), k.transpose(1, 2).contiguous(),
+                 v.transpose(1, 2).contiguous()) for qn, qr, k, v, _ in sets]
     with ctx:
-        calls = [lambda q=q, k=k, v=v: F.scaled_dot_product_attention(q, k, v) for q, k, v in sets]
-        ms = _time_attention_calls(calls, 5)
+        calls = [lambda q=q, k=k, v=v: F.scaled_dot_product_attention(q, k, v) for q, k, v in lib_sets]
+        ms_lib = _time_attention_calls(calls, 5)
     fl = 4.0 * dh * Nq * Nk * d.n_heads
-    del sets
+    del sets, lib_sets
     torch.cuda.empty_cache()
-    return {"what": "torch scaled_dot_product_attention on per-head K / V (library kernel)", "backend": backend,
-            "ms": ms, "tflops": fl / (ms * 1e-3) / 1e12, "cache_bytes_per_token_layer": 2 * 2 * d.n_heads * dh,
-            "latent_cache_bytes_per_token_layer": 2 * (d.d_c + d.d_rope)}
+    return {"what": "dense multi-head attention on per-head K / V, same queries and window",
+            "ours_ms": ms_ours, "ours_tflops": fl / (ms_ours * 1e-3) / 1e12,
+            "library_backend": backend, "library_ms": ms_lib, "library_tflops": fl / (ms_lib * 1e-3) / 1e12,
+            "latent_attention_ms": latent_ms,
+            "latent_over_dense_time": None if latent_ms is None else latent_ms / ms_ours,
+            "cache_bytes_per_token_layer": 2 * 2 * d.n_heads * dh,
+            "latent_cache_bytes_per_token_layer": 2 * (d.d_c + d.d_rope),
+            "dense_window_bytes": 2 * 2 * d.n_heads * dh * Nk, "latent_window_bytes": 2 * (d.d_c + d.d_rope) * Nk}
 
 
 def _graph_time_ms(run, reps: int) -> float:

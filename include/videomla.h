@@ -199,6 +199,27 @@ int videomla_attention_sink(const videomla_dims* dims, const void* q_nope, const
                             size_t workspace_bytes, void* stream);
 
 /*
+ * videomla_dense_attention -- the dense multi-head attention baseline that the
+ * latent cache replaces ("VideoMLA", App. C.1: per-head keys and values cached
+ * for every token, 2 n_h d_h = 3072 scalars per token and layer; Sec. 3.3 Eq. 7),
+ * for same-box comparisons of speed and memory traffic with videomla_attention.
+ * The window's keys are given in logical order (oldest frame first) and the
+ * queries are its newest n_query tokens, with the window-local (t, h, w)
+ * positions of videomla_attention.
+ *   q_nope [batch, n_query, n_heads, d_nope] bf16, q_rope [batch, n_query, n_heads,
+ *          d_rope] bf16 UNROTATED (rotated in the kernel by the query's position).
+ *   k      [batch, n_keys, n_heads, 128] bf16: [k^nope_h | RoPE3D(k^R)], the RoPE part
+ *          already rotated by the key's window-local position.
+ *   v      [batch, n_keys, n_heads, 128] bf16.
+ *   out    [batch, n_query, n_heads, 128] bf16: softmax(q k^T / sqrt(128)) v per head.
+ * Requires d_nope + d_rope == 128, d_v == 128 and n_keys a whole number of frames.
+ * One launch on ``stream``; tcgen05 tensor cores, fp32 online softmax, P as bf16.
+ * Errors: EINVAL (null, sizes, misaligned), EUNSUPPORTED (head widths), ECUDA.
+ */
+int videomla_dense_attention(const videomla_dims* dims, const void* q_nope, const void* q_rope, const void* k,
+                             const void* v, int batch, int n_query, int n_keys, void* out, void* stream);
+
+/*
  * Bytes of the workspace videomla_query_projection needs: the fp32 query latent
  * and its normalised bf16 copy, for batch * n_tok tokens.  0 for invalid arguments.
  */

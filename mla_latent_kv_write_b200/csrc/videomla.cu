@@ -13,6 +13,7 @@
 #include "../../include/videomla.h"
 #include "attention.cuh"
 #include "cache_write.cuh"
+#include "dense_attention.cuh"
 #include "gemm.cuh"
 #include "ptx.cuh"
 
@@ -467,6 +468,58 @@ int run_attention(const videomla_dims* d, const void* q_nope, const void* q_rope
 
 
 // ----------------------------------------------------------------------------
+// dense multi-head attention baseline
+// ----------------------------------------------------------------------------
+template <int DN, int DR>
+int run_dense_attention(const videomla_dims* d, const void* q_nope, const void* q_rope, const void* K, const void* V,
+                        int B, int Nq, int Nk, void* out, cudaStream_t st) {
+    using C = vmla::DenseCfg<DN, DR>;
+    const int H = d->n_heads;
+    vmla::DenseMaps maps;
+    {
+        const uint64_t dims[4] = {uint64_t(C::DH), uint64_t(H), uint64_t(Nk), uint64_t(B)};
+        const uint64_t str[3] = {uint64_t(C::DH) * 2, uint64_t(H) * C::DH * 2, uint64_t(Nk) * H * C::DH * 2};
+        const uint32_t box[4] = {64, 1, uint32_t(C::BK), 1};
+        if (!make_map(&maps.k, K, 4, dims, str, box, 128)) return VIDEOMLA_ECUDA;
+        if (!make_map(&maps.v, V, 4, dims, str, box, 128)) return VIDEOMLA_ECUDA;
+    }
+    vmla::DenseParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.Nq = Nq;
+    p.Nk = Nk;
+    p.H = H;
+    p.T_f = d->grid_h * d->grid_w;
+    p.grid_w = d->grid_w;
+    p.q_first = Nk - Nq;
+    p.n_t = d->pairs_t;
+    p.n_h = d->pairs_h;
+    {
+        // the latent kernel's rope frequencies (an axis owning D_a dims of the head
+        // uses base^(-2k / D_a))
+        const int n_full = (d->d_nope + d->d_rope) / 2;
+        const int full_hw = n_full / 3;
+        const int full_t = n_full - 2 * full_hw;
+        const int cnt[3] = {d->pairs_t, d->pairs_h, d->pairs_w};
+        const int D[3] = {2 * full_t, 2 * full_hw, 2 * full_hw};
+        int pr = 0;
+        for (int a = 0; a < 3; ++a)
+            for (int k = 0; k < cnt[a]; ++k)
+                p.omega[pr++] = float(std::pow(double(d->rope_base), -2.0 * k / double(D[a])));
+    }
+    p.scale_log2 = float(1.4426950408889634 / std::sqrt(double(C::DH)));
+    p.q_nope = static_cast<const __nv_bfloat16*>(q_nope);
+    p.q_rope = static_cast<const __nv_bfloat16*>(q_rope);
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.timeout_ns = g_timeout_ns.load();
+    auto kern = vmla::dense_attention_kernel<C>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+        return VIDEOMLA_ECUDA;
+    dim3 grid((Nq + C::BM - 1) / C::BM, H, B);
+    kern<<<grid, C::THREADS, C::SMEM, st>>>(maps, p);
+    return launch_status(kern, C::SMEM);
+}
+
+// ----------------------------------------------------------------------------
 // projections: C_g [M, N_g] = A [M, K] . B_g [N_g, K]^T, one or two column groups
 // ----------------------------------------------------------------------------
 // Largest number of 2-CTA clusters of a kernel that can be resident at once (cached per device).
@@ -691,6 +744,28 @@ int videomla_attention(const videomla_dims* dims, const void* q_nope, const void
                        void* out, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
     return videomla_attention_sink(dims, q_nope, q_rope, W_uk, W_uv, cache, window, nullptr, 0, batch, n_query, out,
                                    lse, workspace, workspace_bytes, stream);
+}
+
+int videomla_dense_attention(const videomla_dims* dims, const void* q_nope, const void* q_rope, const void* k,
+                             const void* v, int batch, int n_query, int n_keys, void* out, void* stream) {
+    if (!basic_dims_ok(dims) || !q_nope || !q_rope || !k || !v || !out) return VIDEOMLA_EINVAL;
+    if (dims->d_nope + dims->d_rope != 128 || dims->d_v != 128) return VIDEOMLA_EUNSUPPORTED;
+    const long long T_f = (long long)dims->grid_h * dims->grid_w;
+    if (batch <= 0 || batch > 65535 || dims->n_heads > 65535 || n_keys <= 0 || n_keys % T_f != 0 || n_query <= 0 ||
+        n_query > n_keys || (long long)n_keys * dims->n_heads > (1ll << 30))
+        return VIDEOMLA_EINVAL;
+    if (!aligned16(q_nope) || !aligned16(q_rope) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return VIDEOMLA_EINVAL;
+    if (int rc = check_device()) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int dn = dims->d_nope, dr = dims->d_rope;
+#define VMLA_DA(DN_, DR_) \
+    if (dn == DN_ && dr == DR_) return run_dense_attention<DN_, DR_>(dims, q_nope, q_rope, k, v, batch, n_query, n_keys, out, st);
+    VMLA_DA(96, 32)
+    VMLA_DA(112, 16)
+    VMLA_DA(64, 64)
+#undef VMLA_DA
+    return VIDEOMLA_EUNSUPPORTED;
 }
 
 size_t videomla_query_projection_workspace_size(const videomla_dims* dims, int d_q, int batch, int n_tok) {

@@ -32,6 +32,7 @@ EXPORTED = (
     "videomla_attention_sink",
     "videomla_attention_sink_workspace_size",
     "videomla_attention_workspace_size_split",
+    "videomla_dense_attention",
     "videomla_query_projection",
     "videomla_query_projection_workspace_size",
     "videomla_output_projection",
@@ -94,6 +95,8 @@ def load_library() -> ctypes.CDLL:
         lib.videomla_query_projection.argtypes = [ctypes.POINTER(CDims), ci, vp, ci, ci, vp, vp, vp, vp, vp, vp, vp,
                                                   ctypes.c_size_t, vp]
         lib.videomla_query_projection.restype = ci
+        lib.videomla_dense_attention.argtypes = [ctypes.POINTER(CDims), vp, vp, vp, vp, ci, ci, ci, vp, vp]
+        lib.videomla_dense_attention.restype = ci
         lib.videomla_output_projection.argtypes = [ctypes.POINTER(CDims), vp, ci, ci, vp, vp, vp]
         lib.videomla_output_projection.restype = ci
         lib.videomla_strerror.argtypes = [ci]
@@ -289,6 +292,30 @@ def output_projection(o: torch.Tensor, W_O: torch.Tensor, dims: Dims, y: Optiona
     if rc != OK:
         raise VideoMLAError(rc, "videomla_output_projection")
     return y
+
+
+def dense_attention(q_nope: torch.Tensor, q_rope: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dims: Dims,
+                    out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Dense multi-head attention baseline over per-head keys ``k`` and values
+    ``v`` [B, n_keys, H, 128] of a window in logical order (RoPE part of k already
+    rotated); queries are its newest n_query tokens (q_rope unrotated)."""
+    lib = load_library()
+    B, Nq, H = q_nope.shape[0], q_nope.shape[1], dims.n_heads
+    Nk = k.shape[1]
+    dev = q_nope.device
+    _check(q_nope, "q_nope", torch.bfloat16, (B, Nq, H, dims.d_nope))
+    _check(q_rope, "q_rope", torch.bfloat16, (B, Nq, H, dims.d_rope), dev)
+    _check(k, "k", torch.bfloat16, (B, Nk, H, 128), dev)
+    _check(v, "v", torch.bfloat16, (B, Nk, H, 128), dev)
+    if out is None:
+        out = torch.empty(B, Nq, H, 128, dtype=torch.bfloat16, device=dev)
+    _check(out, "out", torch.bfloat16, (B, Nq, H, 128), dev)
+    cd = c_dims(dims)
+    rc = lib.videomla_dense_attention(ctypes.byref(cd), _ptr(q_nope), _ptr(q_rope), _ptr(k), _ptr(v), B, Nq, Nk,
+                                      _ptr(out), _stream(stream))
+    if rc != OK:
+        raise VideoMLAError(rc, "videomla_dense_attention")
+    return out
 
 
 def device_status(reset: bool = False) -> int:

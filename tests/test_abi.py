@@ -118,6 +118,26 @@ def test_valid_call_without_device_reports_no_device(lib):
     assert rc == V.ENODEVICE
 
 
+def test_dense_attention_rejects_bad_arguments(lib):
+    d = _dims()
+    f = lib.videomla_dense_attention
+    T_f = 1560
+    ok_args = [ctypes.byref(d), P, P, P, P, 1, 4680, 21 * T_f, P, None]
+    def call(**over):
+        a = list(ok_args)
+        for i, v in over.items():
+            a[int(i[1:])] = v
+        return f(*a)
+    for i in (1, 2, 3, 4, 8):
+        assert call(**{f"a{i}": None}) == V.EINVAL
+    assert call(a7=21 * T_f + 1) == V.EINVAL              # not a whole number of frames
+    assert call(a6=21 * T_f + 1) == V.EINVAL              # more queries than keys
+    assert call(a6=0) == V.EINVAL
+    assert call(a3=ctypes.c_void_p(0x10008)) == V.EINVAL   # misaligned
+    wide = _dims(); wide.d_v = 192                          # the baseline keeps 128-wide heads
+    assert f(ctypes.byref(wide), *ok_args[1:]) == V.EUNSUPPORTED
+
+
 def test_unsupported_geometry_is_reported(lib):
     import torch
     if not torch.cuda.is_available():
