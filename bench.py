@@ -914,6 +914,30 @@ def profile_sweep(spec: str) -> int:
     return 0
 
 
+def profile_dense() -> int:
+    """Three calls of the dense multi-head attention baseline at the Wan layer
+    shape (random per-head K / V of the 21-frame window), nothing timed: a short
+    command for a profiler to capture one launch of that kernel."""
+    from mla_latent_kv_write_b200 import videomla as V
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    V.load_library()
+    wl, d = WORKLOAD, WORKLOAD.dims
+    Nk = wl.slots * d.tokens_per_frame
+    g = torch.Generator().manual_seed(78)
+    qn = torch.randn(1, wl.n_query, d.n_heads, d.d_nope, generator=g).to(torch.bfloat16).to(dev)
+    qr = torch.randn(1, wl.n_query, d.n_heads, d.d_rope, generator=g).to(torch.bfloat16).to(dev)
+    k = torch.randn(1, Nk, d.n_heads, 128, generator=g).to(torch.bfloat16).to(dev)
+    v = torch.randn(1, Nk, d.n_heads, 128, generator=g).to(torch.bfloat16).to(dev)
+    for _ in range(3):
+        V.dense_attention(qn, qr, k, v, d)
+    torch.cuda.synchronize()
+    if V.device_status(reset=True) != V.OK:
+        raise RuntimeError("a kernel reported a timed-out device wait")
+    print("profile-dense: 3 dense attention calls done")
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -922,11 +946,15 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-side", action="store_true", help="skip the sink-window and sweep side measurements")
+    ap.add_argument("--profile-dense", action="store_true",
+                    help="only run three dense-baseline attention calls (for a profiler), then exit")
     ap.add_argument("--profile-sweep", metavar="D_C,D_ROPE",
                     help="only run three attention calls of one rank-sweep point (for a profiler), then exit")
     args = ap.parse_args()
     if args.profile_sweep:
         return profile_sweep(args.profile_sweep)
+    if args.profile_dense:
+        return profile_dense()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
