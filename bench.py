@@ -614,21 +614,29 @@ def rolling_steps(dev, peak: float):
         q = qs[s % 4]
         V.attention(q["q_nope"], q["q_rope"], w["W_uk"], w["W_uv"], cache, d, wl.slots, oldest, n_valid, out=out)
 
-    for s in range(20):
-        do_step(s)
-    torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for s in range(20, wl.steps):
-        do_step(s)
-    b.record()
-    torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / (wl.steps - 20)
+    def run(mode):
+        with V.attention_tiling(mode):
+            cache.zero_()
+            for s in range(20):
+                do_step(s)
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for s in range(20, wl.steps):
+                do_step(s)
+            b.record()
+            torch.cuda.synchronize()
+        return a.elapsed_time(b) / (wl.steps - 20)
+
+    ms_head = run(V.TILING_PER_HEAD)  # A/B: one CTA per (query tile, head), split-KV over 3 CTAs
+    ms = run(V.TILING_AUTO)           # the library's choice: head-packed tiles
     fl = flops_cache_write(d, wl.batch, T_f) + flops_attention(d, wl.batch, T_f, wl.slots * T_f)
-    ctas = (T_f + 127) // 128 * d.n_heads * wl.batch
+    ctas = (d.n_heads * T_f + 127) // 128 * wl.batch
     return {"workload": "rolling: 1 frame (1560 tokens) per step into a 21-slot ring, steps 20-39 timed",
             "ms_per_step": ms, "tflops": fl / (ms * 1e-3) / 1e12, "frac": fl / (ms * 1e-3) / 1e12 / peak,
-            "attention_ctas": ctas}
+            "attention_ctas": ctas, "tiling": "head-packed (128 consecutive (head, query) rows per CTA)",
+            "per_head_tiles": {"ms_per_step": ms_head, "frac": fl / (ms_head * 1e-3) / 1e12 / peak,
+                               "attention_ctas": "156 units x 3-way split-KV"}}
 
 
 def long_window(dev, peak: float):

@@ -323,6 +323,33 @@ int videomla_device_status(int reset);
 uint64_t videomla_set_wait_timeout_ns(uint64_t ns);
 
 /*
+ * How videomla_attention / videomla_attention_sink assign query rows to CTAs.
+ * Every head attends the same latent keys, so a 128-row tile may hold queries of
+ * two heads: the CTA applies W_uk,h / W_uv,h of each row's own head in its
+ * prologue and epilogue.
+ *   VIDEOMLA_TILING_AUTO         (default) per call, the choice with fewer
+ *                                wave-quantised key-tile times per SM
+ *   VIDEOMLA_TILING_PER_HEAD     one CTA per (128-query tile, head, batch
+ *                                element), key tiles split over up to 4 CTAs
+ *                                when the units leave SMs idle (split-KV)
+ *   VIDEOMLA_TILING_HEAD_PACKED  one CTA per 128 consecutive rows of the
+ *                                head-major (head, query) order of a batch
+ *                                element, never split: 1560 queries x 12 heads
+ *                                take 147 CTAs instead of 156.  Used only where
+ *                                n_query >= 128 and Q stays in tensor memory
+ *                                (d_c + 128 + 64 + (d_c + d_rope) / 2 <= 512);
+ *                                elsewhere the call runs per head.
+ * Process-wide, read at each call.  Every mode computes the same attention; a
+ * row's arithmetic does not depend on the tile that holds it, except that
+ * split-KV merges partial sums.  Returns the previous mode, or VIDEOMLA_EINVAL
+ * (nothing changed) for an unknown mode.
+ */
+#define VIDEOMLA_TILING_AUTO 0
+#define VIDEOMLA_TILING_PER_HEAD 1
+#define VIDEOMLA_TILING_HEAD_PACKED 2
+int videomla_set_attention_tiling(int mode);
+
+/*
  * Self-test of the failure-detection path: launches one CTA that waits, with the
  * same bounded wait the kernels use, on a shared-memory barrier that nothing
  * ever completes.  After ``timeout_ns`` the wait gives up, records

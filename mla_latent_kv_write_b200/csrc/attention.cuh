@@ -58,6 +58,11 @@ struct AttnParams {
     // per-row (max, sum) to part_o / part_ml, and the last of them to arrive
     // (counters, zeroed by the window pre-pass) merges and finishes the unit
     int n_split, tiles_per_split, n_units;
+    // head-packed tiles (never with split-KV): CTA x takes rows [128 x, 128 x + 128)
+    // of the batch element's head-major (head, query) row order, so a tile may end
+    // with the first queries of the next head.  Every head attends the same latent
+    // keys, so only the prologue (W_uk,h) and the epilogue (W_uv,h) see the head.
+    int packed;
     float* part_o;                 // [n_units * n_split, BM, d_c] fp32
     float* part_ml;                // [n_units * n_split, BM, 2] fp32: row max (raw score), row sum
     int* counters;                 // [n_units]
@@ -118,6 +123,9 @@ struct AttnCfg {
     static constexpr int NCH = DC / NMMA;
     static constexpr int O_COL = 0, S_COL = DC, P_COL = DC + BK, Q_COL = DC + BK + BK / 2;
     static constexpr int TMEM_END = QS ? P_COL + BK / 2 : Q_COL + W / 2;
+    // head-packed tiles: the second head's output goes to columns that are idle
+    // once O / l has been staged (O itself, or P and Q when O is narrower)
+    static constexpr int OUT2_COL = DC >= DV ? O_COL : P_COL;
     static constexpr int SMEM = NS * STAGE + QBYTES + 1024 + 1024;
     static constexpr int SM_WARPS_PER_HALF = 4;                 // softmax warps per 16-lane half
     static constexpr int SM_WARPS = 2 * SM_WARPS_PER_HALF;
@@ -127,6 +135,7 @@ struct AttnCfg {
     static_assert(DR == 16 || DR == 32 || DR == 64, "rope width");
     static_assert(DN % 16 == 0 && DV % 32 == 0 && DV <= 256, "head widths");
     static_assert(TMEM_END <= 512 && S_COL + DV <= 512, "tensor memory budget");
+    static_assert(QS || (DC >= DV ? DV <= DC : P_COL + DV <= 512), "second head output region");
     static_assert(SMEM <= 232448 && APS >= 1, "shared memory budget");
     static_assert(QS ? (WUK_OFF + WUK_BYTES <= QBYTES && C_ATOMS * OLAT_ATOM <= QBYTES)
                      : (QN_BYTES <= STAGE && WUK_BYTES <= STAGE && WUV_STAGES == 1 && C_ATOMS * OLAT_ATOM <= STAGE),
@@ -138,6 +147,7 @@ struct AttnBarriers {
     uint64_t part_done, last_known;  // split-KV: partial stored by every softmax warp / arrival counted
     int last_flag, skip_epilogue;
     uint64_t q_full, qabs_done, q_ready, s_full, s_free, p_full, pv_done, olat_ready, out_full, drain, drain2;
+    uint64_t qabs_mid, q2_full, wuv2_full, out2_full;  // head-packed tiles that hold two heads
     uint32_t tmem_base;
     AbortState ab;
 };
@@ -235,10 +245,28 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
     auto stage = [&](int s) { return smem + s * C::STAGE; };
 
     const int warp = warp_id(), lane = lane_id();
-    const int h = blockIdx.y;
     const int b = SPLIT ? int(blockIdx.z) / p.n_split : int(blockIdx.z);
     const int split = SPLIT ? int(blockIdx.z) % p.n_split : 0;
-    const int q0 = blockIdx.x * BM;
+    // Rows r < n1 of the tile are queries i0 + r of head h; with head-packed tiles
+    // rows r >= n1 are queries r - n1 of head h + 1 (a "mixed" tile).
+    const bool packed = !SPLIT && !C::QS && p.packed != 0;
+    int h, i0, n1;
+    if (packed) {
+        const int g0 = int(blockIdx.x) * BM;
+        h = g0 / p.Nq;
+        i0 = g0 - h * p.Nq;
+        n1 = min(BM, p.Nq - i0);
+    } else {
+        h = blockIdx.y;
+        i0 = int(blockIdx.x) * BM;
+        n1 = BM;
+    }
+    const bool mixed = packed && n1 < BM && h + 1 < p.H;
+    auto row_of = [&](int r, int& hr, int& ir) -> bool {  // (head, query) of tile row r; false: no row
+        hr = r < n1 ? h : h + 1;
+        ir = r < n1 ? i0 + r : r - n1;
+        return hr < p.H && ir < p.Nq;
+    };
     const int kt0 = SPLIT ? split * p.tiles_per_split : 0;                       // first key tile of this split
     const int nt = SPLIT ? min(p.n_kt, kt0 + p.tiles_per_split) - kt0 : p.n_kt;  // key tiles of this CTA (>= 1)
     const uint64_t to = p.timeout_ns;
@@ -261,6 +289,10 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
         mbar_init(&bar->drain2, 1);
         mbar_init(&bar->part_done, C::SM_WARPS);
         mbar_init(&bar->last_known, 1);
+        mbar_init(&bar->qabs_mid, 1);
+        mbar_init(&bar->q2_full, 1);
+        mbar_init(&bar->wuv2_full, 1);
+        mbar_init(&bar->out2_full, 1);
         bar->last_flag = 0;
         bar->skip_epilogue = 0;
         ab->flag = 0;
@@ -285,22 +317,36 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
             tma_prefetch_desc(&maps.qn);
             tma_prefetch_desc(&maps.wuk);
             tma_prefetch_desc(&maps.wuv);
-            mbar_arrive_expect_tx(&bar->q_full, C::QN_BYTES + C::WUK_BYTES);
             uint8_t* qn_dst = C::QS ? qreg : stage(NS - 2);
             uint8_t* wuk_dst = C::QS ? qreg + C::WUK_OFF : stage(NS - 1);
-            for (int c = 0; c < C::QN_CHUNKS; ++c)
-                tma_load_4d(qn_dst + c * BM * 32, &maps.qn, &bar->q_full, c * 16, h, q0, b);
-            for (int a = 0; a < C::C_ATOMS; ++a)
-                tma_load_2d(wuk_dst + a * C::WUK_ATOM, &maps.wuk, &bar->q_full, a * 64, h * DN);
+            // q_nope rows of head hh starting at query i (rows past the head's last
+            // query, or before its first, read zeros) and W_uk,hh
+            auto load_q = [&](uint64_t* bq, int hh, int i) {
+                mbar_arrive_expect_tx(bq, C::QN_BYTES + C::WUK_BYTES);
+                for (int c = 0; c < C::QN_CHUNKS; ++c)
+                    tma_load_4d(qn_dst + c * BM * 32, &maps.qn, bq, c * 16, hh, i, b);
+                for (int a = 0; a < C::C_ATOMS; ++a)
+                    tma_load_2d(wuk_dst + a * C::WUK_ATOM, &maps.wuk, bq, a * 64, hh * DN);
+            };
+            load_q(&bar->q_full, h, i0);
+            // mixed tile: once the first q_abs MMAs have read the buffers, the second
+            // head's rows (tile rows n1..127, zeros above them) and W_uk,h+1 replace them
+            bool ok = true, round2 = false, wuv2 = false;
+            auto second_head = [&]() {
+                if (!mixed || round2) return true;
+                if (!mbar_wait(&bar->qabs_mid, 0, ab, to, 12)) return false;
+                load_q(&bar->q2_full, h + 1, -n1);
+                round2 = true;
+                return true;
+            };
             int issued = 0;
             bool qabs_seen = false;
             for (int j = 0; j < nt + C::WUV_STAGES; ++j) {
                 const int s = j % NS;
-                bool ok = true;
                 if (j >= NS) {
                     ok = mbar_wait(&bar->empty[s], ((j / NS) - 1) & 1, ab, to, 10);
                 } else if (!C::QS && s >= NS - 2 && !qabs_seen) {  // stage still holds q_nope / W_uk
-                    ok = qabs_seen = mbar_wait(&bar->qabs_done, 0, ab, to, 11);
+                    ok = second_head() && (qabs_seen = mbar_wait(&bar->qabs_done, 0, ab, to, 11));
                 }
                 if (!ok) break;
                 if (j < nt) {
@@ -319,8 +365,22 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                 }
                 issued = j + 1;
             }
+            ok = ok && second_head();  // a window of fewer tiles never reached stage NS - 2
+            if (ok && mixed) {
+                // W_uv,h+1 into the stage of W_uv,h once the first epilogue MMAs are done
+                ok = mbar_wait(&bar->out_full, 0, ab, to, 13);
+                if (ok) {
+                    mbar_arrive_expect_tx(&bar->wuv2_full, C::C_ATOMS * C::WUV_ATOM);
+                    for (int a = 0; a < C::C_ATOMS; ++a)
+                        tma_load_2d(stage(nt % NS) + a * C::WUV_ATOM, &maps.wuv, &bar->wuv2_full, a * 64,
+                                    (h + 1) * DV);
+                    wuv2 = true;
+                }
+            }
             if (ab->flag) {  // let this CTA's copies land before it exits
                 mbar_wait_drain(&bar->q_full, 0, to);
+                if (round2) mbar_wait_drain(&bar->q2_full, 0, to);
+                if (wuv2) mbar_wait_drain(&bar->wuv2_full, 0, to);
                 for (int j = issued > NS ? issued - NS : 0; j < issued; ++j)
                     mbar_wait_drain(&bar->full[j % NS], (j / NS) & 1, to);
             }
@@ -336,15 +396,31 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                 constexpr uint32_t id_qabs = idesc_bf16_f32(128, C::NCH, false, true);
                 const uint32_t sq = smem_u32(C::QS ? qreg : stage(NS - 2));
                 const uint32_t sw = smem_u32(C::QS ? qreg + C::WUK_OFF : stage(NS - 1));
+                auto qabs_mma = [&](bool acc) {
 #pragma unroll
-                for (int k = 0; k < C::QN_CHUNKS; ++k)
+                    for (int k = 0; k < C::QN_CHUNKS; ++k)
 #pragma unroll
-                    for (int n = 0; n < C::NMMA; ++n)
-                        umma_ss(tmem + C::O_COL + n * C::NCH, sdesc(sq + k * BM * 32, 16, 256, SW32),
-                                sdesc(sw + n * (C::NCH / 64) * C::WUK_ATOM + k * 2048, C::WUK_ATOM, 1024, SW128),
-                                id_qabs, k > 0);
-                umma_commit(&bar->qabs_done);
-                ok = mbar_wait(&bar->q_ready, 0, ab, to, 31);
+                        for (int n = 0; n < C::NMMA; ++n)
+                            umma_ss(tmem + C::O_COL + n * C::NCH, sdesc(sq + k * BM * 32, 16, 256, SW32),
+                                    sdesc(sw + n * (C::NCH / 64) * C::WUK_ATOM + k * 2048, C::WUK_ATOM, 1024, SW128),
+                                    id_qabs, acc || k > 0);
+                };
+                qabs_mma(false);
+                if (mixed) {
+                    // second head: its q_nope rows are zero where the first head's are not
+                    // (and vice versa), so accumulating both products gives each row its own
+                    // head's q_abs exactly
+                    umma_commit(&bar->qabs_mid);
+                    ok = mbar_wait(&bar->q2_full, 0, ab, to, 37);
+                    if (ok) {
+                        tc_fence_after();
+                        qabs_mma(true);
+                    }
+                }
+                if (ok) {
+                    umma_commit(&bar->qabs_done);
+                    ok = mbar_wait(&bar->q_ready, 0, ab, to, 31);
+                }
             }
             constexpr uint32_t id_s = idesc_bf16_f32(128, BK, false, false);
             constexpr uint32_t id_s_rope = idesc_f16_f32(128, BK, false, false);
@@ -391,16 +467,27 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                     constexpr uint32_t id_o = idesc_bf16_f32(128, DV, false, false);
                     const uint32_t ao = smem_u32(C::QS ? qreg : stage((nt + 1) % NS));
                     const uint32_t ao2 = smem_u32(stage((nt + 2) % NS));
+                    auto out_mma = [&](uint32_t col) {
 #pragma unroll
-                    for (int k = 0; k < DC / 16; ++k) {
-                        const int a = k / 4;
-                        const uint32_t bw = smem_u32(stage((nt + a / C::APS) % NS)) + (a % C::APS) * C::WUV_ATOM;
-                        const uint64_t bd = sdesc(bw + (k % 4) * 32, 16, 1024, SW128);
-                        const uint32_t off = a * C::OLAT_ATOM + (k % 4) * 32;
-                        umma_ss(tmem + C::S_COL, sdesc(ao + off, 16, 1024, SW128), bd, id_o, k > 0);
-                        if constexpr (!C::QS) umma_ss(tmem + C::S_COL, sdesc(ao2 + off, 16, 1024, SW128), bd, id_o, 1);
-                    }
+                        for (int k = 0; k < DC / 16; ++k) {
+                            const int a = k / 4;
+                            const uint32_t bw = smem_u32(stage((nt + a / C::APS) % NS)) + (a % C::APS) * C::WUV_ATOM;
+                            const uint64_t bd = sdesc(bw + (k % 4) * 32, 16, 1024, SW128);
+                            const uint32_t off = a * C::OLAT_ATOM + (k % 4) * 32;
+                            umma_ss(tmem + col, sdesc(ao + off, 16, 1024, SW128), bd, id_o, k > 0);
+                            if constexpr (!C::QS) umma_ss(tmem + col, sdesc(ao2 + off, 16, 1024, SW128), bd, id_o, 1);
+                        }
+                    };
+                    out_mma(C::S_COL);
                     umma_commit(&bar->out_full);
+                    if (mixed) {  // the second head's rows: O / l . W_uv,h+1^T into idle columns
+                        ok = mbar_wait(&bar->wuv2_full, 0, ab, to, 38);
+                        if (ok) {
+                            tc_fence_after();
+                            out_mma(C::OUT2_COL);
+                            umma_commit(&bar->out2_full);
+                        }
+                    }
                 }
             }
             if (!ok) {  // no MMA may still run when the tensor memory is released
@@ -473,12 +560,13 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                 }
             }
             if (half == 0) {
-                const int i = q0 + r;
+                int hr, i;
+                const bool has_row = row_of(r, hr, i);
                 uint32_t qr[DR / 2];
 #pragma unroll
                 for (int e = 0; e < DR / 2; ++e) qr[e] = 0u;
-                if (i < p.Nq) {
-                    const uint4* src = reinterpret_cast<const uint4*>(p.q_rope + ((size_t(b) * p.Nq + i) * p.H + h) * DR);
+                if (has_row) {
+                    const uint4* src = reinterpret_cast<const uint4*>(p.q_rope + ((size_t(b) * p.Nq + i) * p.H + hr) * DR);
                     const int L = p.q_first + i;
                     const int tq_ = L / p.T_f;
                     const int pq = L - tq_ * p.T_f;
@@ -819,31 +907,47 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
             if (p.lse != nullptr && quad == 0) {
 #pragma unroll
                 for (int k = 0; k < 2; ++k) {
-                    const int i = q0 + r_top + 8 * k;
-                    if (i < p.Nq)
-                        p.lse[(size_t(b) * p.Nq + i) * p.H + h] = (m_fin[k] * sl + __log2f(l_fin[k])) * 0.69314718055994531f;
+                    int hr, i;
+                    if (row_of(r_top + 8 * k, hr, i))
+                        p.lse[(size_t(b) * p.Nq + i) * p.H + hr] = (m_fin[k] * sl + __log2f(l_fin[k])) * 0.69314718055994531f;
                 }
             }
 
             // out rows of this quadrant, one per thread; the two warps of a quadrant
-            // take alternate 32-column chunks
+            // take alternate 32-column chunks.  A mixed tile's second-head rows read
+            // their own output columns.
             ok = __all_sync(0xffffffffu, mbar_wait(&bar->out_full, 0, ab, to, 45) && !ab->flag);
             if (ok) {
                 tc_fence_after();
-                const int i = q0 + w4 * 32 + lane;
-                __nv_bfloat16* dst = p.out + ((size_t(b) * p.Nq + i) * p.H + h) * DV;
+                const int r = w4 * 32 + lane;
+                int hr, i;
+                const bool has_row = row_of(r, hr, i);
+                const bool second = mixed && r >= n1;
+                __nv_bfloat16* dst = p.out + ((size_t(b) * p.Nq + i) * p.H + hr) * DV;
+                for (int pass = 0; ok && pass < (mixed ? 2 : 1); ++pass) {
+                    const bool mine = second == (pass == 1);
+                    if (!__any_sync(0xffffffffu, mine)) continue;
+                    if (pass == 1) {
+                        ok = __all_sync(0xffffffffu, mbar_wait(&bar->out2_full, 0, ab, to, 48) && !ab->flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                    }
+                    const uint32_t col = pass == 1 ? C::OUT2_COL : C::S_COL;
 #pragma unroll 1
-                for (int c = 32 * half; c < DV; c += 64) {
-                    uint32_t v[32];
-                    tmem_ld_32x32b_x32(tq + C::S_COL + c, v);
-                    tmem_wait_ld();
-                    uint32_t pk[16];
+                    for (int c = 32 * half; c < DV; c += 64) {
+                        uint32_t v[32];
+                        tmem_ld_32x32b_x32(tq + col + c, v);
+                        tmem_wait_ld();
+                        uint32_t pk[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
-                    if (i < p.Nq) {
-                        uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+                        for (int e = 0; e < 16; ++e)
+                            pk[e] = pack_bf16(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+                        if (mine && has_row) {
+                            uint4* d4 = reinterpret_cast<uint4*>(dst + c);
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) d4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                            for (int e = 0; e < 4; ++e)
+                                d4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                        }
                     }
                 }
             }

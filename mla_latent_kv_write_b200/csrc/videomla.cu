@@ -21,6 +21,7 @@ namespace {
 
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
+std::atomic<int> g_tiling{VIDEOMLA_TILING_AUTO};
 
 // ----------------------------------------------------------------------------
 // driver entry point for cuTensorMapEncodeTiled (resolved through the runtime,
@@ -329,24 +330,49 @@ void window_runs(const videomla_window* win, int T_f, int seg_start[3], int seg_
 // tile, head, batch) unit.  One CTA per SM; cost in key-tile times: the waves
 // times the tiles per CTA (+2 for writing a partial), plus the merge of the
 // other partials by the last CTA (1.5 per split).  At most 4 splits.
-int preferred_split(int units, int n_kt, int batch) {
+int attention_sms() {
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
+    return sms > 0 ? sms : 148;
+}
+
+double split_cost(int units, int n_kt, int s, int sms) {
+    const int tps = (n_kt + s - 1) / s;
+    const long long waves = ((long long)units * s + sms - 1) / sms;
+    return double(waves) * (tps + (s > 1 ? 2 : 0)) + 1.5 * (s - 1);
+}
+
+int preferred_split(int units, int n_kt, int batch) {
+    const int sms = attention_sms();
     int best = 1;
     double best_cost = 0;
     for (int s = 1; s <= 4 && s <= n_kt && (long long)batch * s <= 65535; ++s) {
         const int tps = (n_kt + s - 1) / s;
         const int se = (n_kt + tps - 1) / tps;
         if (se != s) continue;
-        const long long waves = ((long long)units * s + sms - 1) / sms;
-        const double cost = double(waves) * (tps + (s > 1 ? 2 : 0)) + 1.5 * (s - 1);
+        const double cost = split_cost(units, n_kt, s, sms);
         if (s == 1 || cost < best_cost) {
             best = s;
             best_cost = cost;
         }
     }
     return best;
+}
+
+// Head-packed query tiles (one CTA per 128 consecutive rows of the head-major
+// (head, query) order, no split-KV) against per-head tiles with their best
+// split: the same wave-count cost, plus ~3 key-tile times for the second
+// head's prologue and epilogue in a tile that holds two heads.  Only for the
+// instances with Q in tensor memory and at least 128 queries (a tile then
+// spans at most two heads).
+bool use_packed_tiles(bool q_in_smem, int Nq, int H, int B, int n_kt, int units, int split) {
+    const int mode = g_tiling.load();
+    if (q_in_smem || Nq < 128 || mode == VIDEOMLA_TILING_PER_HEAD) return false;
+    if (mode == VIDEOMLA_TILING_HEAD_PACKED) return true;
+    const int sms = attention_sms();
+    const long long packed_units = ((long long)H * Nq + 127) / 128 * B;
+    const double packed = double((packed_units + sms - 1) / sms) * n_kt + (Nq % 128 != 0 ? 3.0 : 0.0);
+    return packed < split_cost(units, n_kt, split, sms);
 }
 
 size_t split_part_bytes(int units, int split, int d_c) {  // partial O + (max, sum) per row + counters
@@ -383,6 +409,8 @@ int run_attention(const videomla_dims* d, const void* q_nope, const void* q_rope
         const size_t rope_bytes = align256(size_t(B) * p.ws_rows * DR * 2);
         int sp = preferred_split(units, p.n_kt, B);
         while (sp > 1 && rope_bytes + split_part_bytes(units, sp, DC) > workspace_bytes) --sp;
+        p.packed = use_packed_tiles(C::QS, Nq, H, B, p.n_kt, units, sp) ? 1 : 0;
+        if (p.packed) sp = 1;
         p.tiles_per_split = (p.n_kt + sp - 1) / sp;
         p.n_split = (p.n_kt + p.tiles_per_split - 1) / p.tiles_per_split;
         p.n_units = units;
@@ -461,7 +489,8 @@ int run_attention(const videomla_dims* d, const void* q_nope, const void* q_rope
     auto kern = p.n_split > 1 ? vmla::attention_kernel<C, true> : vmla::attention_kernel<C, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
         return VIDEOMLA_ECUDA;
-    dim3 grid((Nq + C::BM - 1) / C::BM, H, B * p.n_split);
+    const dim3 grid = p.packed ? dim3(unsigned(((long long)H * Nq + C::BM - 1) / C::BM), 1, B)
+                               : dim3((Nq + C::BM - 1) / C::BM, H, B * p.n_split);
     kern<<<grid, C::THREADS, C::SMEM, st>>>(maps, p);
     return launch_status(kern, C::SMEM);
 }
@@ -875,6 +904,12 @@ int videomla_device_status(int reset) {
 
 uint64_t videomla_set_wait_timeout_ns(uint64_t ns) {
     return g_timeout_ns.exchange(ns == 0 ? kDefaultTimeoutNs : ns);
+}
+
+int videomla_set_attention_tiling(int mode) {
+    if (mode != VIDEOMLA_TILING_AUTO && mode != VIDEOMLA_TILING_PER_HEAD && mode != VIDEOMLA_TILING_HEAD_PACKED)
+        return VIDEOMLA_EINVAL;
+    return g_tiling.exchange(mode);
 }
 
 int videomla_selftest_wait_timeout(uint64_t timeout_ns, void* stream) {

@@ -7,6 +7,7 @@ library is missing or cannot be loaded the calls raise: there is no fallback.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import threading
@@ -39,6 +40,7 @@ EXPORTED = (
     "videomla_strerror",
     "videomla_device_status",
     "videomla_set_wait_timeout_ns",
+    "videomla_set_attention_tiling",
     "videomla_selftest_wait_timeout",
     "videomla_version",
 )
@@ -105,6 +107,8 @@ def load_library() -> ctypes.CDLL:
         lib.videomla_device_status.restype = ci
         lib.videomla_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
         lib.videomla_set_wait_timeout_ns.restype = ctypes.c_uint64
+        lib.videomla_set_attention_tiling.argtypes = [ci]
+        lib.videomla_set_attention_tiling.restype = ci
         lib.videomla_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
         lib.videomla_selftest_wait_timeout.restype = ci
         lib.videomla_version.argtypes = []
@@ -324,3 +328,24 @@ def device_status(reset: bool = False) -> int:
 
 def set_wait_timeout_ns(ns: int) -> int:
     return load_library().videomla_set_wait_timeout_ns(ns)
+
+
+TILING_AUTO, TILING_PER_HEAD, TILING_HEAD_PACKED = 0, 1, 2
+
+
+def set_attention_tiling(mode: int) -> int:
+    """Query-row tiling of the attention calls (process-wide); returns the previous mode."""
+    rc = load_library().videomla_set_attention_tiling(mode)
+    if rc < 0:
+        raise VideoMLAError(rc, "videomla_set_attention_tiling")
+    return rc
+
+
+@contextlib.contextmanager
+def attention_tiling(mode: int):
+    """Run the enclosed calls with one tiling mode, then restore the previous one."""
+    prev = set_attention_tiling(mode)
+    try:
+        yield
+    finally:
+        set_attention_tiling(prev)

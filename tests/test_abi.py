@@ -45,6 +45,22 @@ def test_strerror_and_version(lib):
     assert b"unknown" in lib.videomla_strerror(12345)
 
 
+def test_attention_tiling_knob(lib):
+    # header constants and the binding's names agree; unknown modes change nothing
+    hdr = open(os.path.join(ROOT, "include", "videomla.h")).read()
+    for name, val in (("AUTO", V.TILING_AUTO), ("PER_HEAD", V.TILING_PER_HEAD), ("HEAD_PACKED", V.TILING_HEAD_PACKED)):
+        assert re.search(rf"#define VIDEOMLA_TILING_{name} {val}\b", hdr), name
+    assert lib.videomla_set_attention_tiling(V.TILING_PER_HEAD) == V.TILING_AUTO
+    assert lib.videomla_set_attention_tiling(3) == V.EINVAL
+    assert lib.videomla_set_attention_tiling(-1) == V.EINVAL
+    assert lib.videomla_set_attention_tiling(V.TILING_HEAD_PACKED) == V.TILING_PER_HEAD
+    with V.attention_tiling(V.TILING_PER_HEAD):
+        assert lib.videomla_set_attention_tiling(V.TILING_PER_HEAD) == V.TILING_PER_HEAD
+    assert lib.videomla_set_attention_tiling(V.TILING_AUTO) == V.TILING_HEAD_PACKED
+    with pytest.raises(V.VideoMLAError):
+        V.set_attention_tiling(7)
+
+
 def _dims(**kw):
     return V.c_dims(I.Dims(**kw) if kw else I.WAN)
 

@@ -25,14 +25,16 @@ def _dev(d):
     return {k: v.to(DEV) for k, v in d.items()}
 
 
-def _attention_case(dims, B, slots, oldest, n_valid, Nq, seed, rows=None, rope_scale=1.0, n_sink=0):
+def _attention_case(dims, B, slots, oldest, n_valid, Nq, seed, rows=None, rope_scale=1.0, n_sink=0,
+                    tiling=V.TILING_AUTO):
     w = I.layer_weights(dims, seed)
     q = I.queries(dims, B, Nq, seed + 1)
     cache = I.latent_cache(dims, B, slots, seed + 2, rope_scale=rope_scale)
     sink = I.latent_cache(dims, B, n_sink, seed + 3, rope_scale=rope_scale) if n_sink else None
     wd, qd = _dev(w), _dev(q)
-    out, lse = V.attention(qd["q_nope"], qd["q_rope"], wd["W_uk"], wd["W_uv"], cache.to(DEV), dims,
-                           slots, oldest, n_valid, want_lse=True, sink=None if sink is None else sink.to(DEV))
+    with V.attention_tiling(tiling):
+        out, lse = V.attention(qd["q_nope"], qd["q_rope"], wd["W_uk"], wd["W_uv"], cache.to(DEV), dims,
+                               slots, oldest, n_valid, want_lse=True, sink=None if sink is None else sink.to(DEV))
     torch.cuda.synchronize()
     assert V.device_status(reset=True) == V.OK
     ref_out, ref_lse = oracle_attention(dims, q, w, cache, slots, oldest, n_valid, rows, sink_bf16=sink)
@@ -349,9 +351,13 @@ def test_layer_chain_tiny():
 # waves, so the key tiles of each unit are shared by several CTAs
 # ---------------------------------------------------------------------------
 
+# (per-head tiles forced: left to itself the library runs these shapes on
+# head-packed tiles, tested below)
+
 def test_attention_split_kv_sink_window_sampled_rows():
     rows = sample_rows(1560, 48, seed=8)
-    _attention_case(I.WAN, B=1, slots=6, oldest=4, n_valid=6, Nq=1560, seed=1004, rows=rows, n_sink=1)
+    _attention_case(I.WAN, B=1, slots=6, oldest=4, n_valid=6, Nq=1560, seed=1004, rows=rows, n_sink=1,
+                    tiling=V.TILING_PER_HEAD)
 
 
 def test_attention_split_kv_matches_unsplit_call():
@@ -364,10 +370,11 @@ def test_attention_split_kv_matches_unsplit_call():
     cache = I.latent_cache(dims, 1, slots, 1007)
     wd, qd, cd = _dev(w), _dev(q), cache.to(DEV)
     small = torch.empty(V.workspace_size(dims, slots, oldest, slots, 1), dtype=torch.uint8, device=DEV)
-    o1, l1 = V.attention(qd["q_nope"], qd["q_rope"], wd["W_uk"], wd["W_uv"], cd, dims, slots, oldest, slots,
-                         want_lse=True, workspace=small)
-    o2, l2 = V.attention(qd["q_nope"], qd["q_rope"], wd["W_uk"], wd["W_uv"], cd, dims, slots, oldest, slots,
-                         want_lse=True)
+    with V.attention_tiling(V.TILING_PER_HEAD):
+        o1, l1 = V.attention(qd["q_nope"], qd["q_rope"], wd["W_uk"], wd["W_uv"], cd, dims, slots, oldest, slots,
+                             want_lse=True, workspace=small)
+        o2, l2 = V.attention(qd["q_nope"], qd["q_rope"], wd["W_uk"], wd["W_uv"], cd, dims, slots, oldest, slots,
+                             want_lse=True)
     torch.cuda.synchronize()
     assert V.device_status(reset=True) == V.OK
     rows = sample_rows(Nq, 32, seed=9)
@@ -384,7 +391,8 @@ def test_attention_split_kv_batch_two_sampled_rows():
     """1560 queries x 12 heads x batch 2 = 312 units: split over 4 CTAs, so the
     grid's z index carries both the batch element and the split."""
     rows = sample_rows(1560, 24, seed=10)
-    _attention_case(I.WAN, B=2, slots=21, oldest=20, n_valid=21, Nq=1560, seed=1008, rows=rows)
+    _attention_case(I.WAN, B=2, slots=21, oldest=20, n_valid=21, Nq=1560, seed=1008, rows=rows,
+                    tiling=V.TILING_PER_HEAD)
 
 
 def test_attention_split_kv_q_in_shared_memory():
@@ -393,3 +401,62 @@ def test_attention_split_kv_q_in_shared_memory():
     dims = I.sweep_dims(384, 32)
     rows = sample_rows(1560, 24, seed=11)
     _attention_case(dims, B=1, slots=21, oldest=3, n_valid=21, Nq=1560, seed=1009, rows=rows)
+
+
+# ---------------------------------------------------------------------------
+# head-packed tiles: a CTA takes 128 consecutive rows of the head-major (head,
+# query) order, so a tile may end with the first queries of the next head
+# ("mixed"): its q_abs comes from two accumulated MMAs over zero-padded q_nope
+# boxes, its output from a second W_uv MMA into other tensor-memory columns
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("slots,oldest,n_valid,Nq,B,n_sink", [
+    (7, 4, 5, 200, 2, 0),   # 19 tiles per batch element, 11 of them mixed; wrapped ring, ragged key tiles
+    (7, 0, 7, 130, 1, 0),   # each head's last 2 queries start a tile; 13 tiles
+    (5, 2, 3, 144, 2, 0),   # 144 keys, two key tiles: the W_uv load is the first to reuse a q_nope / W_uk stage
+    (6, 4, 6, 144, 1, 1),   # sink frame + wrapping FIFO: three runs of key rows
+    (7, 3, 7, 336, 1, 0),   # 32 tiles, the last one ragged (the last head's rows end inside it)
+])
+def test_attention_head_packed_tiles(slots, oldest, n_valid, Nq, B, n_sink):
+    _attention_case(I.TINY, B=B, slots=slots, oldest=oldest, n_valid=n_valid, Nq=Nq, seed=6100 + Nq + slots,
+                    n_sink=n_sink, tiling=V.TILING_HEAD_PACKED)
+
+
+@pytest.mark.parametrize("d_c,d_rope", [(96, 32), (192, 16), (192, 64)])
+def test_attention_head_packed_sweep_points(d_c, d_rope):
+    # d_c = 96: the second head's output sits in the P / Q columns (O is narrower
+    # than d_v); (192, 64): 3 ring stages
+    dims = dataclasses.replace(I.sweep_dims(d_c, d_rope), grid_h=6, grid_w=8)
+    _attention_case(dims, B=2, slots=5, oldest=3, n_valid=4, Nq=150, seed=6300 + d_c + d_rope,
+                    tiling=V.TILING_HEAD_PACKED)
+
+
+def test_attention_rolling_shape_head_packed_sampled_rows():
+    """The rolling step's attention: 1560 queries x 12 heads over the full
+    21-frame ring, which the library runs on 147 head-packed CTAs (one wave)."""
+    rows = sample_rows(1560, 48, seed=12)
+    _attention_case(I.WAN, B=1, slots=21, oldest=5, n_valid=21, Nq=1560, seed=6400, rows=rows)
+
+
+@pytest.mark.parametrize("dims,slots,oldest,n_valid,Nq,B", [
+    (I.TINY, 7, 4, 5, 200, 2),
+    (I.WAN, 21, 0, 21, 1560, 1),
+])
+def test_attention_head_packed_equals_per_head(dims, slots, oldest, n_valid, Nq, B):
+    """A row's arithmetic does not depend on the tile that holds it: head-packed
+    and unsplit per-head tiles give the same bits (the per-head call gets a
+    workspace with no room for split-KV partials)."""
+    w = _dev(I.layer_weights(dims, 6500))
+    q = _dev(I.queries(dims, B, Nq, 6501))
+    cache = I.latent_cache(dims, B, slots, 6502).to(DEV)
+    small = torch.empty(V.workspace_size(dims, slots, oldest, n_valid, B), dtype=torch.uint8, device=DEV)
+    outs = []
+    for mode in (V.TILING_PER_HEAD, V.TILING_HEAD_PACKED):
+        with V.attention_tiling(mode):
+            outs.append(V.attention(q["q_nope"], q["q_rope"], w["W_uk"], w["W_uv"], cache, dims, slots, oldest,
+                                    n_valid, want_lse=True, workspace=small))
+    torch.cuda.synchronize()
+    assert V.device_status(reset=True) == V.OK
+    (o1, l1), (o2, l2) = outs
+    assert torch.equal(o1, o2)
+    assert torch.equal(l1, l2)
