@@ -12,6 +12,7 @@
 
 #include "../../include/videomla.h"
 #include "attention.cuh"
+#include "attention_pp.cuh"
 #include "cache_write.cuh"
 #include "dense_attention.cuh"
 #include "gemm.cuh"
@@ -419,6 +420,19 @@ int run_attention(const videomla_dims* d, const void* q_nope, const void* q_rope
         p.part_ml = p.part_o + size_t(units) * p.n_split * 128 * DC;
         p.counters = reinterpret_cast<int*>(p.part_ml + size_t(units) * p.n_split * 128 * 2);
     }
+    // Narrow latents without split-KV or head-packed tiles run the two-group kernel,
+    // whose key tiles are shorter: recount them and size the key maps' boxes for it.
+    bool two_group = false;
+    int bk = C::BK;
+    if constexpr (vmla::pingpong_fits(DC)) {
+        two_group = p.n_split == 1 && !p.packed;
+        if (two_group) {
+            bk = vmla::AttnPPCfg<DC, DR, DN, DV>::BK;
+            p.n_kt = 0;
+            for (int r = 0; r < 3; ++r) p.n_kt += (p.seg_len[r] + bk - 1) / bk;
+            p.tiles_per_split = p.n_kt;
+        }
+    }
     p.q_first = (n_sink + win->n_valid) * T_f - Nq;
     p.n_t = d->pairs_t;
     p.n_h = d->pairs_h;
@@ -452,12 +466,12 @@ int run_attention(const videomla_dims* d, const void* q_nope, const void* q_rope
         const uint64_t batch_rows = is_sink ? uint64_t(n_sink) * T_f : uint64_t(rows);
         const uint64_t dc[3] = {uint64_t(C::W), uint64_t(p.seg_len[run]), uint64_t(B)};
         const uint64_t sc[2] = {uint64_t(C::W) * 2, batch_rows * C::W * 2};
-        const uint32_t bc[3] = {64, uint32_t(C::BK), 1};
+        const uint32_t bc[3] = {64, uint32_t(bk), 1};
         if (!make_map(&maps.cc[r], base, 3, dc, sc, bc, 128)) return VIDEOMLA_ECUDA;
         const size_t ws_row0 = is_sink ? size_t(rows) : size_t(p.seg_start[run]);
         const uint64_t dr[3] = {uint64_t(DR), uint64_t(p.seg_len[run]), uint64_t(B)};
         const uint64_t sr[2] = {uint64_t(DR) * 2, uint64_t(p.ws_rows) * DR * 2};
-        const uint32_t br[3] = {uint32_t(DR), uint32_t(C::BK), 1};
+        const uint32_t br[3] = {uint32_t(DR), uint32_t(bk), 1};
         if (!make_map(&maps.kr[r], krot + ws_row0 * DR, 3, dr, sr, br, DR * 2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
             return VIDEOMLA_ECUDA;
     }
@@ -486,6 +500,16 @@ int run_attention(const videomla_dims* d, const void* q_nope, const void* q_rope
         vmla::rope_window_kernel<DC, DR><<<blocks, 256, 0, st>>>(cache_b, sink_b, static_cast<__half*>(workspace), p, B);
     }
     // 2) latent attention
+    if constexpr (vmla::pingpong_fits(DC)) {
+        if (two_group) {
+            using PC = vmla::AttnPPCfg<DC, DR, DN, DV>;
+            auto kern = vmla::attention_pp_kernel<PC>;
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PC::SMEM) != cudaSuccess)
+                return VIDEOMLA_ECUDA;
+            kern<<<dim3((Nq + PC::BM - 1) / PC::BM, H, B), PC::THREADS, PC::SMEM, st>>>(maps, p);
+            return launch_status(kern, PC::SMEM);
+        }
+    }
     auto kern = p.n_split > 1 ? vmla::attention_kernel<C, true> : vmla::attention_kernel<C, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
         return VIDEOMLA_ECUDA;

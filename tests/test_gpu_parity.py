@@ -460,3 +460,29 @@ def test_attention_head_packed_equals_per_head(dims, slots, oldest, n_valid, Nq,
     (o1, l1), (o2, l2) = outs
     assert torch.equal(o1, o2)
     assert torch.equal(l1, l2)
+
+
+# ---------------------------------------------------------------------------
+# d_c = 96: two softmax groups on alternate key tiles, each with its own S
+# buffer, O accumulator and running (max, sum), merged at the end
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("slots,oldest,n_valid,Nq,B,n_sink,rope_scale", [
+    (5, 2, 1, 48, 1, 0, 1.0),    # one key tile: the second group has no tile at all
+    (5, 1, 2, 96, 2, 0, 1.0),    # 96 keys, still one (ragged) tile
+    (5, 3, 3, 144, 1, 0, 1.0),   # two tiles, the second ragged: one per group
+    (7, 4, 5, 200, 2, 0, 1.0),   # wrapped ring, two runs with ragged tiles, 3 tiles (odd count)
+    (7, 2, 7, 200, 1, 0, 8.0),   # peaky scores: the stale-max rescale of each group's O
+    (6, 4, 6, 144, 2, 1, 1.0),   # sink frame + wrapping FIFO: three runs of key rows
+])
+def test_attention_two_group_narrow_latent(slots, oldest, n_valid, Nq, B, n_sink, rope_scale):
+    dims = dataclasses.replace(I.sweep_dims(96, 32), grid_h=6, grid_w=8)
+    _attention_case(dims, B=B, slots=slots, oldest=oldest, n_valid=n_valid, Nq=Nq, seed=6600 + 7 * slots + Nq,
+                    rope_scale=rope_scale, n_sink=n_sink, tiling=V.TILING_PER_HEAD)
+
+
+def test_attention_two_group_narrow_latent_wan_window_sampled_rows():
+    """d_c = 96 at the Wan shape (256 key tiles: 128 per group), sampled rows."""
+    dims = I.sweep_dims(96, 32)
+    rows = sample_rows(4680, 48, seed=13)
+    _attention_case(dims, B=1, slots=21, oldest=9, n_valid=21, Nq=4680, seed=6700, rows=rows)
