@@ -357,13 +357,16 @@ __global__ void __launch_bounds__(352, 1) attention_pp_kernel(const __grid_const
                     for (int c = 0; c < 32; ++c)
                         if (32 * q + c >= valid) sv[q][c] = 0xff800000u;  // -inf
             }
-            float mxq[NQ];
+            float mxq[NQ];  // two independent max chains per 32-column chunk
 #pragma unroll
             for (int q = 0; q < NQ; ++q) {
-                float m = __uint_as_float(sv[q][0]);
+                float m0 = __uint_as_float(sv[q][0]), m1 = __uint_as_float(sv[q][16]);
 #pragma unroll
-                for (int c = 1; c < 31; c += 2) m = fmax3(m, __uint_as_float(sv[q][c]), __uint_as_float(sv[q][c + 1]));
-                mxq[q] = fmaxf(m, __uint_as_float(sv[q][31]));
+                for (int c = 1; c < 15; c += 2) {
+                    m0 = fmax3(m0, __uint_as_float(sv[q][c]), __uint_as_float(sv[q][c + 1]));
+                    m1 = fmax3(m1, __uint_as_float(sv[q][16 + c]), __uint_as_float(sv[q][16 + c + 1]));
+                }
+                mxq[q] = fmaxf(fmax3(m0, m1, __uint_as_float(sv[q][15])), __uint_as_float(sv[q][31]));
             }
             float mx = mxq[0];
 #pragma unroll
@@ -384,19 +387,22 @@ __global__ void __launch_bounds__(352, 1) attention_pp_kernel(const __grid_const
             // P = exp2(s sl - m sl) as bf16 pairs: column c of P_g holds keys 2c, 2c + 1
             const float2 sl2 = make_float2(sl, sl);
             const float2 nm = make_float2(-m_used * sl, -m_used * sl);
-            float2 acc = make_float2(0.f, 0.f);
+            float2 acc[NQ];  // one row-sum chain per chunk
             uint32_t pk[NQ][16];
 #pragma unroll
-            for (int q = 0; q < NQ; ++q)
+            for (int q = 0; q < NQ; ++q) {
+                acc[q] = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int c = 0; c < 16; ++c) {
                     const float2 x = __ffma2_rn(
                         make_float2(__uint_as_float(sv[q][2 * c]), __uint_as_float(sv[q][2 * c + 1])), sl2, nm);
                     const float2 e = make_float2(ex2(x.x), ex2(x.y));
-                    acc = __fadd2_rn(acc, e);
+                    acc[q] = __fadd2_rn(acc[q], e);
                     pk[q][c] = pack_bf16(e.x, e.y);
                 }
-            l_run += acc.x + acc.y;
+            }
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) l_run += acc[q].x + acc[q].y;
             // P_g and O_g are free once this group's previous PV has completed
             if (k >= 1) {
                 ok = __all_sync(0xffffffffu, mbar_wait(&bar->pv_done[g], (k - 1) & 1, ab, to, 72));
