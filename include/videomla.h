@@ -283,11 +283,13 @@ int videomla_output_projection(const videomla_dims* dims, const void* o, int bat
  * - Sizes: if videomla_attention_workspace_size(dims, window, batch) exceeds
  *   VIDEOMLA_STATIC_WORKSPACE_BYTES the call returns VIDEOMLA_EINVAL and
  *   launches nothing.  When the preferred split's partials do not fit beside
- *   the RoPE keys the call runs with the largest split that fits, or unsplit:
- *   the 1560-query Wan frame step (156 units, 2-4 splits of 31-62 MB) runs
- *   unsplit here, a few query tiles against a long window (e.g. 128 queries,
- *   12 heads, 21 Wan frames: 4.8 MB of partials) keep their split.  Results
- *   agree with videomla_attention to rounding either way.
+ *   the RoPE keys the call runs with the largest split that fits, or unsplit,
+ *   or on head-packed tiles (videomla_set_attention_tiling) where those need
+ *   fewer waves: the 1560-query Wan frame step (156 per-head units) runs on
+ *   147 head-packed CTAs here as in videomla_attention; a few query tiles
+ *   against a long window (e.g. 128 queries, 12 heads, 21 Wan frames: 4.8 MB
+ *   of partials) keep their split.  Results agree with videomla_attention to
+ *   rounding either way.
  * - Set-up: every call looks up the device address of the scratch array in the
  *   current context (cudaGetSymbolAddress); the first such lookup on a device
  *   may load the library's kernels, so make the first call before any stream
