@@ -121,6 +121,13 @@ struct AttnCfg {
     // MMAs of N = DC (q_abs, P C) run as NMMA column halves of NCH <= 256
     static constexpr int NMMA = DC > 256 ? 2 : 1;
     static constexpr int NCH = DC / NMMA;
+    // With Q in shared memory only two ring stages fit, so each stage is filled and
+    // freed in two halves: latent blocks [0, LO_ATOMS) ("lo") and the rest with the
+    // rotated RoPE keys ("hi").  The two N halves of the PV MMA are their last
+    // readers, so a stage's lo half refills while PV still reads its hi half, and
+    // the next score MMAs start on the lo blocks before the hi half has landed.
+    static constexpr bool HALVES = QS && NMMA == 2 && C_ATOMS % 2 == 0;
+    static constexpr int LO_ATOMS = HALVES ? C_ATOMS / 2 : C_ATOMS;
     static constexpr int O_COL = 0, S_COL = DC, P_COL = DC + BK, Q_COL = DC + BK + BK / 2;
     static constexpr int TMEM_END = QS ? P_COL + BK / 2 : Q_COL + W / 2;
     // head-packed tiles: the second head's output goes to columns that are idle
@@ -132,6 +139,7 @@ struct AttnCfg {
     static constexpr int THREADS = 32 * (3 + SM_WARPS);
     static_assert(DC % 32 == 0 && NCH % 64 == 0 || NMMA == 1, "latent width");
     static_assert(DC % 32 == 0 && NCH <= 256, "latent width");
+    static_assert(!HALVES || NCH / 64 == LO_ATOMS, "PV half n reads latent blocks [n LO_ATOMS, (n + 1) LO_ATOMS)");
     static_assert(DR == 16 || DR == 32 || DR == 64, "rope width");
     static_assert(DN % 16 == 0 && DV % 32 == 0 && DV <= 256, "head widths");
     static_assert(TMEM_END <= 512 && S_COL + DV <= 512, "tensor memory budget");
@@ -144,6 +152,7 @@ struct AttnCfg {
 
 struct AttnBarriers {
     uint64_t full[4], empty[4];
+    uint64_t full_hi[4], empty_hi[4];  // the hi halves of the stages (HALVES only)
     uint64_t part_done, last_known;  // split-KV: partial stored by every softmax warp / arrival counted
     int last_flag, skip_epilogue;
     uint64_t q_full, qabs_done, q_ready, s_full, s_free, p_full, pv_done, olat_ready, out_full, drain, drain2;
@@ -275,6 +284,8 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
         for (int s = 0; s < NS; ++s) {
             mbar_init(&bar->full[s], 1);
             mbar_init(&bar->empty[s], 1);
+            mbar_init(&bar->full_hi[s], 1);
+            mbar_init(&bar->empty_hi[s], 1);
         }
         mbar_init(&bar->q_full, 1);
         mbar_init(&bar->qabs_done, 1);
@@ -352,11 +363,23 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                 if (j < nt) {
                     int run, row, valid;
                     key_tile<BK>(p, kt0 + j, run, row, valid);
-                    mbar_arrive_expect_tx(&bar->full[s], C::STAGE);
-                    for (int a = 0; a < C::C_ATOMS; ++a)
+                    uint64_t* fh = C::HALVES ? &bar->full_hi[s] : &bar->full[s];  // barrier of the hi half
+                    mbar_arrive_expect_tx(&bar->full[s], C::HALVES ? C::LO_ATOMS * C::C_ATOM : C::STAGE);
+                    for (int a = 0; a < C::LO_ATOMS; ++a)
                         tma_load_3d(stage(s) + a * C::C_ATOM, &maps.cc[run], &bar->full[s], a * 64, row, b);
-                    tma_load_3d(stage(s) + C::C_ATOMS * C::C_ATOM, &maps.kr[run], &bar->full[s], 0, row, b);
+                    if constexpr (C::HALVES) {
+                        if (j >= NS) ok = mbar_wait(&bar->empty_hi[s], ((j / NS) - 1) & 1, ab, to, 14);
+                        if (!ok) break;
+                        mbar_arrive_expect_tx(fh, C::STAGE - C::LO_ATOMS * C::C_ATOM);
+                    }
+                    for (int a = C::LO_ATOMS; a < C::C_ATOMS; ++a)
+                        tma_load_3d(stage(s) + a * C::C_ATOM, &maps.cc[run], fh, a * 64, row, b);
+                    tma_load_3d(stage(s) + C::C_ATOMS * C::C_ATOM, &maps.kr[run], fh, 0, row, b);
                 } else {  // W_uv blocks [a0, a1) of the epilogue
+                    if constexpr (C::HALVES) {
+                        if (j >= NS) ok = mbar_wait(&bar->empty_hi[s], ((j / NS) - 1) & 1, ab, to, 15);
+                        if (!ok) break;
+                    }
                     const int a0 = (j - nt) * C::APS;
                     const int a1 = a0 + C::APS < C::C_ATOMS ? a0 + C::APS : C::C_ATOMS;
                     mbar_arrive_expect_tx(&bar->full[s], (a1 - a0) * C::WUV_ATOM);
@@ -381,8 +404,10 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                 mbar_wait_drain(&bar->q_full, 0, to);
                 if (round2) mbar_wait_drain(&bar->q2_full, 0, to);
                 if (wuv2) mbar_wait_drain(&bar->wuv2_full, 0, to);
-                for (int j = issued > NS ? issued - NS : 0; j < issued; ++j)
+                for (int j = issued > NS ? issued - NS : 0; j < issued; ++j) {
                     mbar_wait_drain(&bar->full[j % NS], (j / NS) & 1, to);
+                    if (C::HALVES && j < nt) mbar_wait_drain(&bar->full_hi[j % NS], (j / NS) & 1, to);
+                }
             }
         }
     } else if (warp == 1) {
@@ -435,9 +460,18 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                 if constexpr (C::QS) {
                     const uint32_t sq = smem_u32(qreg);
 #pragma unroll
-                    for (int k = 0; k < DC / 16; ++k)
+                    for (int k = 0; k < DC / 16; ++k) {
+                        if (C::HALVES && k == C::LO_ATOMS * 4) {  // the hi half of the stage
+                            if (!mbar_wait(&bar->full_hi[s], (j / NS) & 1, ab, to, 39)) break;
+                            tc_fence_after();
+                        }
                         umma_ss(tmem + C::S_COL, sdesc(sq + (k / 4) * C::Q_ATOM + (k % 4) * 32, 16, 1024, SW128),
                                 sdesc(st + (k / 4) * C::C_ATOM + (k % 4) * 32, 16, 1024, SW128), id_s, k > 0);
+                    }
+                    if (ab->flag) {
+                        ok = false;
+                        break;
+                    }
 #pragma unroll
                     for (int k = 0; k < DR / 16; ++k)
                         umma_ss(tmem + C::S_COL, sdesc(sq + C::QR_OFF + k * 32, 16, 8 * C::R_ROWB, C::R_SW),
@@ -507,13 +541,15 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                 tc_fence_after();
                 const uint32_t st = smem_u32(stage(sp));
 #pragma unroll
-                for (int k = 0; k < BK / 16; ++k)
+                for (int n = 0; n < C::NMMA; ++n) {
 #pragma unroll
-                    for (int n = 0; n < C::NMMA; ++n)
+                    for (int k = 0; k < BK / 16; ++k)
                         umma_ts(tmem + C::O_COL + n * C::NCH, tmem + C::P_COL + k * 8,
                                 sdesc(st + n * (C::NCH / 64) * C::C_ATOM + k * 2048, C::C_ATOM, 1024, SW128), id_pv,
                                 (jj > 0 || k > 0));
-                umma_commit(&bar->empty[sp]);
+                    if (C::HALVES) umma_commit(n == 0 ? &bar->empty[sp] : &bar->empty_hi[sp]);
+                }
+                if (!C::HALVES) umma_commit(&bar->empty[sp]);
                 umma_commit(&bar->pv_done);
             }
             umma_commit(&bar->drain2);
