@@ -129,7 +129,12 @@ struct AttnCfg {
     static constexpr bool HALVES = QS && NMMA == 2 && C_ATOMS % 2 == 0;
     static constexpr int LO_ATOMS = HALVES ? C_ATOMS / 2 : C_ATOMS;
     static constexpr int O_COL = 0, S_COL = DC, P_COL = DC + BK, Q_COL = DC + BK + BK / 2;
-    static constexpr int TMEM_END = QS ? P_COL + BK / 2 : Q_COL + W / 2;
+    // With Q in shared memory the score tile is double-buffered: S_j in columns
+    // S_COL + (j mod 2) BK, and P_j (bf16 pairs) over the first BK / 2 columns of
+    // its own S buffer, so the next tile's score MMAs need not wait for the
+    // softmax; S_{j+2} is issued once PV_j has read P_j.
+    static constexpr bool S2 = QS;
+    static constexpr int TMEM_END = QS ? S_COL + 2 * BK : Q_COL + W / 2;
     // head-packed tiles: the second head's output goes to columns that are idle
     // once O / l has been staged (O itself, or P and Q when O is narrower)
     static constexpr int OUT2_COL = DC >= DV ? O_COL : P_COL;
@@ -153,6 +158,8 @@ struct AttnCfg {
 struct AttnBarriers {
     uint64_t full[4], empty[4];
     uint64_t full_hi[4], empty_hi[4];  // the hi halves of the stages (HALVES only)
+    uint64_t pv_buf[2];                // PV of a tile whose P sits in S buffer b (S2 only)
+    uint64_t s_full2[2];               // S_j complete in buffer j % 2 (S2 only)
     uint64_t part_done, last_known;  // split-KV: partial stored by every softmax warp / arrival counted
     int last_flag, skip_epilogue;
     uint64_t q_full, qabs_done, q_ready, s_full, s_free, p_full, pv_done, olat_ready, out_full, drain, drain2;
@@ -292,6 +299,10 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
         mbar_init(&bar->q_ready, C::SM_WARPS);
         mbar_init(&bar->s_full, 1);
         mbar_init(&bar->s_free, C::SM_WARPS);
+        mbar_init(&bar->pv_buf[0], 1);
+        mbar_init(&bar->pv_buf[1], 1);
+        mbar_init(&bar->s_full2[0], 1);
+        mbar_init(&bar->s_full2[1], 1);
         mbar_init(&bar->p_full, C::SM_WARPS);
         mbar_init(&bar->pv_done, 1);
         mbar_init(&bar->olat_ready, C::SM_WARPS);
@@ -453,10 +464,15 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                 // S_j = Q . K_j^T : K = DC latent (bf16) + DR rotated rope (fp16) columns
                 const int s = j % NS;
                 ok = mbar_wait(&bar->full[s], (j / NS) & 1, ab, to, 32);
-                if (ok && j > 0) ok = mbar_wait(&bar->s_free, (j - 1) & 1, ab, to, 33);
+                if constexpr (C::S2) {  // S buffer j % 2 holds P_{j-2} until PV_{j-2} has read it
+                    if (ok && j >= 2) ok = mbar_wait(&bar->pv_buf[j & 1], ((j - 2) >> 1) & 1, ab, to, 33);
+                } else {
+                    if (ok && j > 0) ok = mbar_wait(&bar->s_free, (j - 1) & 1, ab, to, 33);
+                }
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t st = smem_u32(stage(s));
+                const uint32_t s_col = C::S_COL + (C::S2 ? (j & 1) * BK : 0);
                 if constexpr (C::QS) {
                     const uint32_t sq = smem_u32(qreg);
 #pragma unroll
@@ -465,7 +481,7 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                             if (!mbar_wait(&bar->full_hi[s], (j / NS) & 1, ab, to, 39)) break;
                             tc_fence_after();
                         }
-                        umma_ss(tmem + C::S_COL, sdesc(sq + (k / 4) * C::Q_ATOM + (k % 4) * 32, 16, 1024, SW128),
+                        umma_ss(tmem + s_col, sdesc(sq + (k / 4) * C::Q_ATOM + (k % 4) * 32, 16, 1024, SW128),
                                 sdesc(st + (k / 4) * C::C_ATOM + (k % 4) * 32, 16, 1024, SW128), id_s, k > 0);
                     }
                     if (ab->flag) {
@@ -474,7 +490,7 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                     }
 #pragma unroll
                     for (int k = 0; k < DR / 16; ++k)
-                        umma_ss(tmem + C::S_COL, sdesc(sq + C::QR_OFF + k * 32, 16, 8 * C::R_ROWB, C::R_SW),
+                        umma_ss(tmem + s_col, sdesc(sq + C::QR_OFF + k * 32, 16, 8 * C::R_ROWB, C::R_SW),
                                 sdesc(st + C::C_ATOMS * C::C_ATOM + k * 32, 16, 8 * C::R_ROWB, C::R_SW), id_s_rope, 1);
                 } else {
 #pragma unroll
@@ -486,7 +502,7 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                         umma_ts(tmem + C::S_COL, tmem + C::Q_COL + DC / 2 + k * 8,
                                 sdesc(st + C::C_ATOMS * C::C_ATOM + k * 32, 16, 8 * C::R_ROWB, C::R_SW), id_s_rope, 1);
                 }
-                umma_commit(&bar->s_full);
+                umma_commit(C::S2 ? &bar->s_full2[j & 1] : &bar->s_full);
             }
             if (ok) {
                 // out [128 x DV] = O_lat [128 x DC] . W_uv,h^T  (all K-major SW128).  With Q in
@@ -540,16 +556,18 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t st = smem_u32(stage(sp));
+                const uint32_t p_col = C::S2 ? C::S_COL + (jj & 1) * BK : C::P_COL;
 #pragma unroll
                 for (int n = 0; n < C::NMMA; ++n) {
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)
-                        umma_ts(tmem + C::O_COL + n * C::NCH, tmem + C::P_COL + k * 8,
+                        umma_ts(tmem + C::O_COL + n * C::NCH, tmem + p_col + k * 8,
                                 sdesc(st + n * (C::NCH / 64) * C::C_ATOM + k * 2048, C::C_ATOM, 1024, SW128), id_pv,
                                 (jj > 0 || k > 0));
                     if (C::HALVES) umma_commit(n == 0 ? &bar->empty[sp] : &bar->empty_hi[sp]);
                 }
                 if (!C::HALVES) umma_commit(&bar->empty[sp]);
+                if (C::S2) umma_commit(&bar->pv_buf[jj & 1]);
                 umma_commit(&bar->pv_done);
             }
             umma_commit(&bar->drain2);
@@ -647,13 +665,15 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
         //   (columns 8k + 2 quad + {0, 1} of each 64-column half of the tile).
         float m_used[2] = {0.f, 0.f}, l_part[2] = {0.f, 0.f};
         for (int j = 0; ok && j < nt; ++j) {
-            ok = __all_sync(0xffffffffu, mbar_wait(&bar->s_full, j & 1, ab, to, 41));
+            ok = __all_sync(0xffffffffu, C::S2 ? mbar_wait(&bar->s_full2[j & 1], (j >> 1) & 1, ab, to, 41)
+                                               : mbar_wait(&bar->s_full, j & 1, ab, to, 41));
             if (!ok) break;
             tc_fence_after();
             constexpr int NC = BK / 64;  // 64-column halves of the tile
             uint32_t sv[NC][32];
+            const uint32_t s_col = C::S_COL + (C::S2 ? (j & 1) * BK : 0);
 #pragma unroll
-            for (int c = 0; c < NC; ++c) tmem_ld_16x256b_x8(tb + C::S_COL + 64 * c, sv[c]);
+            for (int c = 0; c < NC; ++c) tmem_ld_16x256b_x8(tb + s_col + 64 * c, sv[c]);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
@@ -761,15 +781,18 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                 }
             l_part[0] += acc0.x + acc0.y;
             l_part[1] += acc1.x + acc1.y;
-            if (j > 0 && !waited) {  // P_{j-1} must have been consumed before P_j overwrites it
+            if (!C::S2 && j > 0 && !waited) {  // P_{j-1} must have been consumed before P_j overwrites it
                 ok = __all_sync(0xffffffffu, mbar_wait(&bar->pv_done, (j - 1) & 1, ab, to, 43));
                 if (!ok) break;
                 tc_fence_after();
             }
+            // (S2: P_j goes over this tile's own scores, already in registers; PV_{j-2},
+            // the last reader of that buffer, completed before S_j was issued)
+            const uint32_t p_col = C::S2 ? s_col : C::P_COL;
             if constexpr (NC == 2) {
-                tmem_st_16x128b_x16(tb + C::P_COL, pa);
+                tmem_st_16x128b_x16(tb + p_col, pa);
             } else {
-                tmem_st_16x128b_x8(tb + C::P_COL, pa);
+                tmem_st_16x128b_x8(tb + p_col, pa);
             }
             tmem_wait_st();
             tc_fence_before();
