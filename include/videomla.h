@@ -149,6 +149,11 @@ size_t videomla_attention_workspace_size_split(const videomla_dims* dims, const 
  *          videomla_attention_workspace_size_split() bytes also the split-KV
  *          partials).  Calls that run concurrently need distinct workspaces.
  * Two launches on ``stream``: the window pre-pass, then the attention kernel.
+ * The kernel's CTAs take 128 query rows each: of one head (split-KV when those
+ * units leave SMs idle), or 128 consecutive rows of the head-major (head, query)
+ * order when that needs fewer waves (videomla_set_attention_tiling).  The d_c = 96
+ * instance, when it runs neither split-KV nor head-packed tiles, uses two softmax
+ * warpgroups on alternate 96-key tiles, merged exactly at the end.
  * Arithmetic: tcgen05 tensor cores with fp32 accumulation; the latent part of
  * the scores uses bf16 operands (q_abs rounded to bf16), the RoPE part fp16
  * operands (rotated q^R and k^R), the probabilities are rounded to bf16 before
