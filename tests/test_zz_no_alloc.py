@@ -3,8 +3,9 @@
 Some callers cannot hand the library a scratch buffer: their device memory is
 owned by a pool or arena they do not expose, or they run where a cudaMalloc is
 not allowed.  ``videomla_attention_static_workspace`` serves them with a scratch
-array compiled into the library.  This test calls it through the C ABI three
-times in a row, on different windows (one of them split-KV), and checks each
+array compiled into the library.  This test calls it through the C ABI four
+times in a row, on different windows (one split-KV, one on head-packed query
+tiles), and checks each
 result against the regular ``videomla_attention`` (caller workspace) on the same
 inputs, with the tolerance the other attention tests use.  It also checks that
 a window too large for the built-in array is refused before anything is
@@ -59,10 +60,12 @@ def test_static_workspace_matches_regular_entry_point_in_a_row():
         # against the same 21-frame window, which splits its key tiles 4 ways
         # with the partials and counters in the array behind the RoPE keys, on
         # top of what the first call left there; then a wrapped tiny window with
-        # ragged tiles and batch 2: no call may see another's rows
+        # ragged tiles and batch 2: no call may see another's rows; last the
+        # 1560-query frame step, which runs on 147 head-packed CTAs
         (I.WAN, 1, 21, 0, 21, 4680, 31, False),
         (I.WAN, 1, 21, 5, 21, 128, 33, True),
         (I.TINY, 2, 7, 4, 5, 100, 32, None),
+        (I.WAN, 1, 21, 9, 21, 1560, 34, None),
     ]
     for dims, B, slots, oldest, n_valid, Nq, seed, splits in cases:
         rope = V.workspace_size(dims, slots, oldest, n_valid, B)
