@@ -972,6 +972,28 @@ def profile_dense() -> int:
     return 0
 
 
+def profile_projection() -> int:
+    """Three calls of the output projection (W_O over the 12 heads' outputs) at
+    the Wan chunk shape (4680 tokens), nothing timed: a short command for a
+    profiler to capture one launch of the pair GEMM."""
+    from mla_latent_kv_write_b200 import videomla as V
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    V.load_library()
+    d, M = WORKLOAD.dims, WORKLOAD.n_query
+    pw = {n: t.to(dev) for n, t in I.projection_weights(d, 77).items()}
+    g = torch.Generator().manual_seed(79)
+    o = torch.randn(1, M, d.n_heads, d.d_v, generator=g).to(torch.bfloat16).to(dev)
+    y = torch.empty(1, M, d.d_model, dtype=torch.bfloat16, device=dev)
+    for _ in range(3):
+        V.output_projection(o, pw["W_O"], d, y=y)
+    torch.cuda.synchronize()
+    if V.device_status(reset=True) != V.OK:
+        raise RuntimeError("a kernel reported a timed-out device wait")
+    print("profile-projection: 3 output projection calls done")
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -980,6 +1002,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-side", action="store_true", help="skip the sink-window and sweep side measurements")
+    ap.add_argument("--profile-projection", action="store_true",
+                    help="only run three output-projection calls at the Wan shape (for a profiler), then exit")
     ap.add_argument("--profile-dense", action="store_true",
                     help="only run three dense-baseline attention calls (for a profiler), then exit")
     ap.add_argument("--profile-sweep", metavar="D_C,D_ROPE",
@@ -989,6 +1013,8 @@ def main():
         return profile_sweep(args.profile_sweep)
     if args.profile_dense:
         return profile_dense()
+    if args.profile_projection:
+        return profile_projection()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
