@@ -231,8 +231,11 @@ int main(void) {
     d.grid_h = 30; d.grid_w = 52; d.pairs_t = 6; d.pairs_h = 5; d.pairs_w = 5;
     d.rope_base = 10000.0f; d.rms_eps = 1e-6f;
     w.slots = 21; w.oldest_slot = 0; w.n_valid = 21;
-    printf("%d|%s|%zu\n", videomla_version(), videomla_strerror(VIDEOMLA_EINVAL),
-           videomla_attention_workspace_size(&d, &w, 1));
+    int prev = videomla_set_attention_tiling(VIDEOMLA_TILING_HEAD_PACKED);
+    int back = videomla_set_attention_tiling(prev);
+    int bad = videomla_set_attention_tiling(99);
+    printf("%d|%s|%zu|%d|%d|%d\n", videomla_version(), videomla_strerror(VIDEOMLA_EINVAL),
+           videomla_attention_workspace_size(&d, &w, 1), prev, back, bad);
     return 0;
 }
 """
@@ -257,7 +260,9 @@ def test_plain_c_caller_links_and_calls_host_entry_points(lib):
     subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"), src,
                     "-L", pkg, "-lvideomla", "-Wl,-rpath," + pkg, "-o", exe], check=True)
     r = subprocess.run([exe], check=True, capture_output=True, text=True)
-    version, err, ws = r.stdout.strip().split("|")
+    version, err, ws, prev, back, bad = r.stdout.strip().split("|")
     assert int(version) == lib.videomla_version()
     assert err == lib.videomla_strerror(V.EINVAL).decode()
     assert int(ws) == 21 * 1560 * 32 * 2
+    # a fresh process starts in automatic tiling; setting returns the previous mode
+    assert (int(prev), int(back), int(bad)) == (V.TILING_AUTO, V.TILING_HEAD_PACKED, V.EINVAL)
