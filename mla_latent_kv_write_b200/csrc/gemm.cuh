@@ -17,9 +17,9 @@
 //              N BN, K 16 steps); two accumulators, so the next tile's MMAs run
 //              while the epilogues drain this one
 //   warps 2-5  epilogue: one TMEM lane (row of C) per thread, 16-byte stores
-//              of the columns below N
-// rms_norm_rows_kernel: one warp per row of an fp32 [M, D] matrix, bf16 output
-// g * v / sqrt(mean(v^2) + eps).
+//              of the columns below N; optionally a per-row sum of squares
+//              (atomically added), a per-column scale and a per-row 1 / rms
+//              scale, which together carry the query path's RMSNorm
 #pragma once
 
 #include "ptx.cuh"
@@ -35,6 +35,14 @@ struct GemmParams {
     void* C[2];           // [M, ldc] bf16 or fp32, row-major
     int ldc[2];           // elements
     uint64_t timeout_ns;
+    // optional epilogue work (RMSNorm split across two GEMMs): row_ss[row] += sum of
+    // the row's squared fp32 outputs; column c scaled by col_scale[c]; every row
+    // scaled by 1 / sqrt(row_ss_in[row] / rms_dim + rms_eps)
+    float* row_ss;
+    const float* col_scale;
+    const float* row_ss_in;
+    int rms_dim;
+    float rms_eps;
 };
 
 // Tile index -> (row tile, column group, first column in the group).
@@ -188,11 +196,31 @@ __global__ void __launch_bounds__(192, 1)
             const int row = m0 + r;
             const int N = g == 0 ? p.N[0] : p.N[1], ldc = g == 0 ? p.ldc[0] : p.ldc[1];
             void* const Cg = g == 0 ? p.C[0] : p.C[1];
+            const float rscale = p.row_ss_in != nullptr && row < p.M
+                                     ? rsqrtf(__ldg(p.row_ss_in + row) / float(p.rms_dim) + p.rms_eps)
+                                     : 1.0f;
+            float ss = 0.f;
 #pragma unroll 1
             for (int c = 0; c < BN; c += 32) {
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(trow + c, v);
                 tmem_wait_ld();
+                if (p.row_ss != nullptr) {  // columns past N are zeros (B rows past N read zeros)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) ss = fmaf(__uint_as_float(v[e]), __uint_as_float(v[e]), ss);
+                }
+                if (p.col_scale != nullptr || p.row_ss_in != nullptr) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4) {
+                        float4 cs = make_float4(1.f, 1.f, 1.f, 1.f);
+                        if (p.col_scale != nullptr && n0 + c + e + 4 <= N)
+                            cs = __ldg(reinterpret_cast<const float4*>(p.col_scale + n0 + c + e));
+                        v[e + 0] = __float_as_uint(__uint_as_float(v[e + 0]) * cs.x * rscale);
+                        v[e + 1] = __float_as_uint(__uint_as_float(v[e + 1]) * cs.y * rscale);
+                        v[e + 2] = __float_as_uint(__uint_as_float(v[e + 2]) * cs.z * rscale);
+                        v[e + 3] = __float_as_uint(__uint_as_float(v[e + 3]) * cs.w * rscale);
+                    }
+                }
                 if (row < p.M) {
                     if constexpr (C::F32OUT) {
                         float* dst = static_cast<float*>(Cg) + size_t(row) * ldc + n0 + c;
@@ -215,6 +243,7 @@ __global__ void __launch_bounds__(192, 1)
                     }
                 }
             }
+            if (p.row_ss != nullptr && row < p.M) atomicAdd(p.row_ss + row, ss);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {  // the accumulator may take tile j + 2 (rank 0's barrier counts both CTAs)
@@ -230,34 +259,6 @@ __global__ void __launch_bounds__(192, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc_pair(tmem, C::TMEM_COLS);
-    }
-}
-
-// out[m, :] = bf16(g * in[m, :] / sqrt(mean(in[m, :]^2) + eps)), D % 4 == 0; one warp per row.
-__global__ void __launch_bounds__(256) rms_norm_rows_kernel(const float* __restrict__ in, __nv_bfloat16* __restrict__ out,
-                                                            const float* __restrict__ gamma, int M, int D, float eps) {
-    const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (row >= M) return;
-    const float* src = in + size_t(row) * D;
-    float ss = 0.f;
-    for (int c = lane * 4; c < D; c += 128) {
-        const float4 v = *reinterpret_cast<const float4*>(src + c);
-        ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float scale = rsqrtf(ss / float(D) + eps);
-    __nv_bfloat16* dst = out + size_t(row) * D;
-    for (int c = lane * 4; c < D; c += 128) {
-        const float4 v = *reinterpret_cast<const float4*>(src + c);
-        float g0 = 1.f, g1 = 1.f, g2 = 1.f, g3 = 1.f;
-        if (gamma != nullptr) {
-            const float4 g = *reinterpret_cast<const float4*>(gamma + c);
-            g0 = g.x; g1 = g.y; g2 = g.z; g3 = g.w;
-        }
-        *reinterpret_cast<uint2*>(dst + c) =
-            make_uint2(pack_bf16(v.x * scale * g0, v.y * scale * g1), pack_bf16(v.z * scale * g2, v.w * scale * g3));
     }
 }
 

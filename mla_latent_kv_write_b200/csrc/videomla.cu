@@ -607,9 +607,18 @@ int max_pair_clusters(const void* kern, int threads, int smem) {
     return n;
 }
 
+// Optional epilogue work of a GEMM launch (see GemmParams).
+struct GemmEpilogue {
+    float* row_ss = nullptr;
+    const float* col_scale = nullptr;
+    const float* row_ss_in = nullptr;
+    int rms_dim = 1;
+    float rms_eps = 0.f;
+};
+
 template <int BN, bool F32OUT>
 int run_gemm_pair(const void* A, int M, int K, int groups, const void* B0, int N0, void* C0, int ldc0, const void* B1,
-                  int N1, void* C1, int ldc1, cudaStream_t st) {
+                  int N1, void* C1, int ldc1, cudaStream_t st, const GemmEpilogue& epi) {
     using C = vmla::GemmPairCfg<BN, F32OUT>;
     CUtensorMap ta, tb[2];
     {
@@ -645,6 +654,11 @@ int run_gemm_pair(const void* A, int M, int K, int groups, const void* B0, int N
     p.ldc[0] = ldc0;
     p.ldc[1] = ldc1;
     p.timeout_ns = g_timeout_ns.load();
+    p.row_ss = epi.row_ss;
+    p.col_scale = epi.col_scale;
+    p.row_ss_in = epi.row_ss_in;
+    p.rms_dim = epi.rms_dim;
+    p.rms_eps = epi.rms_eps;
     const int pairs_max = max_pair_clusters(reinterpret_cast<const void*>(kern), C::THREADS, C::SMEM);
     const int pairs = p.tiles < pairs_max ? p.tiles : pairs_max;
     cudaLaunchConfig_t cfg = {};
@@ -683,16 +697,17 @@ int gemm_pair_bn(int M, int N0, int N1, int groups) {
 
 // bf16 or fp32 C; one or two column groups sharing A; CTA-pair kernel.
 int gemm2(const void* A, int M, int K, int groups, const void* B0, int N0, void* C0, int ldc0, const void* B1, int N1,
-          void* C1, int ldc1, bool f32out, cudaStream_t st) {
+          void* C1, int ldc1, bool f32out, cudaStream_t st, const GemmEpilogue& epi = GemmEpilogue()) {
     if (gemm_pair_bn(M, N0, N1, groups) == 256)
-        return f32out ? run_gemm_pair<256, true>(A, M, K, groups, B0, N0, C0, ldc0, B1, N1, C1, ldc1, st)
-                      : run_gemm_pair<256, false>(A, M, K, groups, B0, N0, C0, ldc0, B1, N1, C1, ldc1, st);
-    return f32out ? run_gemm_pair<128, true>(A, M, K, groups, B0, N0, C0, ldc0, B1, N1, C1, ldc1, st)
-                  : run_gemm_pair<128, false>(A, M, K, groups, B0, N0, C0, ldc0, B1, N1, C1, ldc1, st);
+        return f32out ? run_gemm_pair<256, true>(A, M, K, groups, B0, N0, C0, ldc0, B1, N1, C1, ldc1, st, epi)
+                      : run_gemm_pair<256, false>(A, M, K, groups, B0, N0, C0, ldc0, B1, N1, C1, ldc1, st, epi);
+    return f32out ? run_gemm_pair<128, true>(A, M, K, groups, B0, N0, C0, ldc0, B1, N1, C1, ldc1, st, epi)
+                  : run_gemm_pair<128, false>(A, M, K, groups, B0, N0, C0, ldc0, B1, N1, C1, ldc1, st, epi);
 }
 
-int gemm(const void* A, const void* B, int M, int N, int K, void* Cmat, int ldc, bool f32out, cudaStream_t st) {
-    return gemm2(A, M, K, 1, B, N, Cmat, ldc, nullptr, 0, nullptr, 0, f32out, st);
+int gemm(const void* A, const void* B, int M, int N, int K, void* Cmat, int ldc, bool f32out, cudaStream_t st,
+         const GemmEpilogue& epi = GemmEpilogue()) {
+    return gemm2(A, M, K, 1, B, N, Cmat, ldc, nullptr, 0, nullptr, 0, f32out, st, epi);
 }
 
 }  // namespace
@@ -824,7 +839,7 @@ int videomla_dense_attention(const videomla_dims* dims, const void* q_nope, cons
 size_t videomla_query_projection_workspace_size(const videomla_dims* dims, int d_q, int batch, int n_tok) {
     if (!dims || d_q <= 0 || batch <= 0 || n_tok <= 0) return 0;
     const size_t m = size_t(batch) * n_tok;
-    return align256(m * d_q * 4) + m * d_q * 2;
+    return align256(m * 4) + m * d_q * 2;  // per-row sums of squares, then g (.) c^Q in bf16
 }
 
 int videomla_query_projection(const videomla_dims* dims, int d_q, const void* x, int batch, int n_tok,
@@ -842,14 +857,23 @@ int videomla_query_projection(const videomla_dims* dims, int d_q, const void* x,
         return VIDEOMLA_EINVAL;
     if (int rc = check_device()) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    float* cq = static_cast<float*>(workspace);
-    auto* cqn = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(workspace) + align256(size_t(M) * d_q * 4));
-    // c^Q = x W_dq^T (fp32), RMSNorm -> bf16, then the two up-projections
-    if (int rc = gemm(x, W_dq, int(M), d_q, dims->d_model, cq, d_q, true, st)) return rc;
-    vmla::rms_norm_rows_kernel<<<int((M + 7) / 8), 256, 0, st>>>(cq, cqn, gamma_q, int(M), d_q, dims->rms_eps);
-    if (cudaGetLastError() != cudaSuccess) return VIDEOMLA_ECUDA;
-    // both up-projections read the normalised c^Q: one launch, two column groups
-    return gemm2(cqn, int(M), d_q, 2, W_uq, int(nq), q_nope, int(nq), W_qr, int(nr), q_rope, int(nr), false, st);
+    // RMSNorm(c^Q) = g (.) c^Q / rms(c^Q) is linear in g (.) c^Q up to the per-row factor, so it
+    // is split over the two GEMMs: the first writes g (.) c^Q (bf16) and adds each row's sum
+    // of squares of c^Q (fp32, before g and rounding); the second, both up-projections in
+    // one launch (two column groups), scales its output rows by 1 / rms.
+    float* ss = static_cast<float*>(workspace);
+    auto* cqg = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(workspace) + align256(size_t(M) * 4));
+    if (cudaMemsetAsync(ss, 0, size_t(M) * 4, st) != cudaSuccess) return VIDEOMLA_ECUDA;
+    GemmEpilogue first;
+    first.row_ss = ss;
+    first.col_scale = gamma_q;
+    if (int rc = gemm(x, W_dq, int(M), d_q, dims->d_model, cqg, d_q, false, st, first)) return rc;
+    GemmEpilogue second;
+    second.row_ss_in = ss;
+    second.rms_dim = d_q;
+    second.rms_eps = dims->rms_eps;
+    return gemm2(cqg, int(M), d_q, 2, W_uq, int(nq), q_nope, int(nq), W_qr, int(nr), q_rope, int(nr), false, st,
+                 second);
 }
 
 int videomla_output_projection(const videomla_dims* dims, const void* o, int batch, int n_query, const void* W_O,
