@@ -280,15 +280,17 @@ def _norm_rel(got, ref):
     return float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
 
 
-@pytest.mark.parametrize("dims,n_tok,B,rows", [
-    (I.TINY, 144, 2, None),
-    (I.WAN, 4680, 1, "sample"),
+@pytest.mark.parametrize("dims,n_tok,B,rows,unit_gain", [
+    (I.TINY, 144, 2, None, False),
+    (I.TINY, 144, 1, None, True),     # gamma_q = NULL: the GEMM epilogue applies no column gain
+    (I.WAN, 4680, 1, "sample", False),
 ])
-def test_query_projection(dims, n_tok, B, rows):
-    pw = I.projection_weights(dims, 610, random_gamma=True)
+def test_query_projection(dims, n_tok, B, rows, unit_gain):
+    pw = I.projection_weights(dims, 610, random_gamma=not unit_gain)
     x = I.tokens(dims, B, n_tok, 611)
     d = _dev(pw)
-    qn, qr = V.query_projection(x.to(DEV), d["W_dq"], d["gamma_q"], d["W_uq"], d["W_qr"], dims)
+    qn, qr = V.query_projection(x.to(DEV), d["W_dq"], None if unit_gain else d["gamma_q"], d["W_uq"], d["W_qr"],
+                                dims)
     torch.cuda.synchronize()
     assert V.device_status(reset=True) == V.OK
     sel = np.arange(n_tok) if rows is None else sample_rows(n_tok, 64, seed=612)
