@@ -29,6 +29,12 @@
  *     validated and enqueued.  A kernel whose bounded device-side wait ran out
  *     records VIDEOMLA_ETIMEOUT in a device status word, read with
  *     videomla_device_status().
+ *   - Stream order holds as for any kernel.  The attention, its window pre-pass
+ *     and the projection GEMMs are launched with programmatic stream
+ *     serialisation: their CTAs may start (barriers, tensor memory, query
+ *     loads) while the previous kernel of the stream drains, and they wait for
+ *     that kernel to finish before reading anything it may have written or
+ *     writing anything.
  *   - Errors are returned as negative codes (below); no exception crosses the
  *     ABI and nothing is printed.  videomla_strerror() names a code.
  *   - Thread safety: calls may be made from several host threads; the only

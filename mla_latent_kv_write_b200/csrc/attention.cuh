@@ -206,6 +206,11 @@ __global__ void __launch_bounds__(256) rope_window_kernel(const __nv_bfloat16* _
                                                           const __nv_bfloat16* __restrict__ sink,
                                                           __half* __restrict__ krot, const AttnParams p, int B) {
     constexpr int W = DC + DR, CH = DR / 8;
+    // Launched programmatically: nothing is read before the previous kernel has
+    // finished.  Only then may the attention start: its prologue reads queries
+    // that kernel (or an earlier one) may have written, and nothing of ours.
+    griddep_wait();
+    griddep_launch_dependents();
     if (p.n_split > 1) {  // arrival counters of the split-KV attention launched next
         for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < p.n_units;
              i += (long long)gridDim.x * blockDim.x)
@@ -259,6 +264,7 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
     AttnBarriers* bar = reinterpret_cast<AttnBarriers*>(qreg + C::QBYTES);
     AbortState* ab = &bar->ab;
     auto stage = [&](int s) { return smem + s * C::STAGE; };
+    griddep_launch_dependents();  // every CTA of this grid is resident or done before a dependent starts
 
     const int warp = warp_id(), lane = lane_id();
     const int b = SPLIT ? int(blockIdx.z) / p.n_split : int(blockIdx.z);
@@ -351,6 +357,11 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
                     tma_load_2d(wuk_dst + a * C::WUK_ATOM, &maps.wuk, bq, a * 64, hh * DN);
             };
             load_q(&bar->q_full, h, i0);
+            // Launched programmatically after the RoPE pre-pass, which lets it start
+            // only once every kernel before the pass has finished: the queries and
+            // W_uk are complete; the window (and the split counters the pass
+            // clears) are read only after the pass has finished too.
+            griddep_wait();
             // mixed tile: once the first q_abs MMAs have read the buffers, the second
             // head's rows (tile rows n1..127, zeros above them) and W_uk,h+1 replace them
             bool ok = true, round2 = false, wuv2 = false;
@@ -659,6 +670,8 @@ __global__ void __launch_bounds__(352, 1) attention_kernel(const __grid_constant
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar->q_ready);
         }
+
+        griddep_wait();  // the stores below may not overtake the RoPE pre-pass
 
         // main loop.  16x256b layout: this thread holds rows
         //   R0 = w4*32 + half*16 + lane/4 and R1 = R0 + 8, 32 columns of each

@@ -90,6 +90,7 @@ __global__ void __launch_bounds__(352, 1) attention_pp_kernel(const __grid_const
     auto stage = [&](int s) { return smem + s * C::STAGE; };
     uint8_t* olat_hi = smem;                 // epilogue: O / l in bf16 hi and lo parts over the
     uint8_t* olat_lo = smem + C::OLAT_BYTES;  // first stages, idle once every PV MMA has completed
+    griddep_launch_dependents();  // every CTA of this grid is resident or done before a dependent starts
 
     const int warp = warp_id(), lane = lane_id();
     const int h = blockIdx.y, b = blockIdx.z;
@@ -146,6 +147,7 @@ __global__ void __launch_bounds__(352, 1) attention_pp_kernel(const __grid_const
                 tma_load_4d(stage(NS - 2) + c * BM * 32, &maps.qn, &bar->q_full, c * 16, h, q0, b);
             for (int a = 0; a < C::C_ATOMS; ++a)
                 tma_load_2d(stage(NS - 1) + a * C::WUK_ATOM, &maps.wuk, &bar->q_full, a * 64, h * DN);
+            griddep_wait();  // the window is read only after the RoPE pre-pass has finished
             int issued = 0;
             bool qabs_seen = false, ok = true, wuv = false;
             for (int j = 0; j < nt; ++j) {
@@ -330,6 +332,8 @@ __global__ void __launch_bounds__(352, 1) attention_pp_kernel(const __grid_const
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar->q_ready);
         }
+
+        griddep_wait();  // the stores below may not overtake the RoPE pre-pass
 
         // main loop over this group's tiles j = g, g + 2, ...; one row per thread,
         // register c of chunk q = score column 32 q + c

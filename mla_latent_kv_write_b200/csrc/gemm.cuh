@@ -96,6 +96,7 @@ __global__ void __launch_bounds__(192, 1)
     const int pair = int(blockIdx.x) >> 1, P = int(gridDim.x) >> 1;
     const int k_chunks = p.K / BK;
     const uint64_t to = p.timeout_ns;
+    griddep_launch_dependents();  // the grid is persistent: all of it is resident from the start
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
@@ -118,6 +119,9 @@ __global__ void __launch_bounds__(192, 1)
     cluster_sync();  // both CTAs' barriers exist before any cross-CTA arrive or byte count
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // Launched programmatically: the set-up above overlaps the previous kernel's
+    // tail; no thread touches global memory before that kernel has finished.
+    griddep_wait();
     auto stage_a = [&](int s) { return smem + s * C::STAGE; };
     auto stage_b = [&](int s) { return smem + s * C::STAGE + C::A_BYTES; };
 

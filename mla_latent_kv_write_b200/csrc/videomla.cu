@@ -100,6 +100,25 @@ int launch_status(K kernel, int smem) {
     return e == cudaSuccess ? VIDEOMLA_OK : VIDEOMLA_ECUDA;
 }
 
+// Launch with programmatic stream serialisation: the kernel may start while the
+// previous kernel of the stream drains, and it calls griddep_wait before it
+// touches anything that kernel writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_programmatic(void (*kern)(KArgs...), dim3 grid, int threads, int smem, cudaStream_t st,
+                                Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 bool basic_dims_ok(const videomla_dims* d) {
     if (!d) return false;
     if (d->d_model <= 0 || d->n_heads <= 0 || d->d_c <= 0 || d->d_rope <= 0 || d->d_nope <= 0 || d->d_v <= 0)
@@ -497,7 +516,11 @@ int run_attention(const videomla_dims* d, const void* q_nope, const void* q_rope
     {
         const long long work = (long long)B * (p.seg_len[0] + p.seg_len[1] + p.seg_len[2]) * (DR / 8);
         const int blocks = int((work + 255) / 256);
-        vmla::rope_window_kernel<DC, DR><<<blocks, 256, 0, st>>>(cache_b, sink_b, static_cast<__half*>(workspace), p, B);
+        if (launch_programmatic(vmla::rope_window_kernel<DC, DR>, dim3(blocks), 256, 0, st, cache_b, sink_b,
+                                static_cast<__half*>(workspace), p, B) != cudaSuccess) {
+            cudaGetLastError();
+            return VIDEOMLA_ECUDA;
+        }
     }
     // 2) latent attention
     if constexpr (vmla::pingpong_fits(DC)) {
@@ -506,7 +529,13 @@ int run_attention(const videomla_dims* d, const void* q_nope, const void* q_rope
             auto kern = vmla::attention_pp_kernel<PC>;
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PC::SMEM) != cudaSuccess)
                 return VIDEOMLA_ECUDA;
-            kern<<<dim3((Nq + PC::BM - 1) / PC::BM, H, B), PC::THREADS, PC::SMEM, st>>>(maps, p);
+            // launched right behind the pre-pass, which lets it start only once all
+            // kernels before the pass have finished
+            if (launch_programmatic(kern, dim3((Nq + PC::BM - 1) / PC::BM, H, B), PC::THREADS, PC::SMEM, st, maps,
+                                    p) != cudaSuccess) {
+                cudaGetLastError();
+                return VIDEOMLA_ECUDA;
+            }
             return launch_status(kern, PC::SMEM);
         }
     }
@@ -515,7 +544,10 @@ int run_attention(const videomla_dims* d, const void* q_nope, const void* q_rope
         return VIDEOMLA_ECUDA;
     const dim3 grid = p.packed ? dim3(unsigned(((long long)H * Nq + C::BM - 1) / C::BM), 1, B)
                                : dim3((Nq + C::BM - 1) / C::BM, H, B * p.n_split);
-    kern<<<grid, C::THREADS, C::SMEM, st>>>(maps, p);
+    if (launch_programmatic(kern, grid, C::THREADS, C::SMEM, st, maps, p) != cudaSuccess) {
+        cudaGetLastError();
+        return VIDEOMLA_ECUDA;
+    }
     return launch_status(kern, C::SMEM);
 }
 
@@ -666,13 +698,15 @@ int run_gemm_pair(const void* A, int M, int K, int groups, const void* B0, int N
     cfg.blockDim = dim3(C::THREADS);
     cfg.dynamicSmemBytes = C::SMEM;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // set-up overlaps the previous kernel
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     if (cudaLaunchKernelEx(&cfg, kern, ta, tb[0], tb[1], p) != cudaSuccess) {
         cudaGetLastError();
         return VIDEOMLA_ECUDA;
