@@ -231,8 +231,9 @@ int videomla_dense_attention(const videomla_dims* dims, const void* q_nope, cons
                              const void* v, int batch, int n_query, int n_keys, void* out, void* stream);
 
 /*
- * Bytes of the workspace videomla_query_projection needs: a per-token fp32 sum of
- * squares of the query latent and the latent times its gain in bf16, for
+ * Bytes of the workspace videomla_query_projection needs: per token, up to
+ * ceil(d_q / 128) fp32 partial sums of squares of the query latent (one per
+ * column tile of the first GEMM), and the latent times its gain in bf16, for
  * batch * n_tok tokens.  0 for invalid arguments.
  */
 size_t videomla_query_projection_workspace_size(const videomla_dims* dims, int d_q, int batch, int n_tok);
@@ -242,16 +243,18 @@ size_t videomla_query_projection_workspace_size(const videomla_dims* dims, int d
  * Sec. 3.1 Eq. 3-4, Sec. 3.2 Eq. 6, App. D.2):
  *   c^Q = W_dq x (fp32), RMSNorm with gain gamma_q and dims->rms_eps (App. D.2),
  *   q_nope = W_uq c^Q and q_rope = W_qr c^Q (unrotated; videomla_attention rotates it).
- *   The RMSNorm is carried by the GEMMs: the first stores gamma_q (.) c^Q in bf16 and
- *   sums each token's squares of c^Q in fp32, the second scales its output rows by
- *   1 / sqrt(mean square + rms_eps) before rounding them to bf16.
+ *   The RMSNorm is carried by the GEMMs: the first stores gamma_q (.) c^Q in bf16 and,
+ *   for each of its column tiles, the sum of each token's squares of c^Q in fp32; the
+ *   second adds a token's partial sums (in tile order, so the result does not depend
+ *   on scheduling) and scales its output rows by 1 / sqrt(mean square + rms_eps)
+ *   before rounding them to bf16.
  *   x       [batch, n_tok, d_model] bf16
  *   W_dq    [d_q, d_model] bf16; gamma_q [d_q] fp32 or NULL (unit gain)
  *   W_uq    [n_heads * d_nope, d_q] bf16, W_qr [n_heads * d_rope, d_q] bf16
  *   q_nope  [batch, n_tok, n_heads, d_nope] bf16, q_rope [batch, n_tok, n_heads, d_rope] bf16
  *   workspace  at least videomla_query_projection_workspace_size() bytes, 16-byte aligned.
- * A memset of the sums of squares and two persistent tcgen05 GEMM launches (the
- * second writes both up-projections) on ``stream``.
+ * Two persistent tcgen05 GEMM launches (the second writes both up-projections) on
+ * ``stream``; the workspace needs no initialisation.
  * Errors: EINVAL (null, d_q or d_model not a multiple of 64, n_heads * d_nope or
  * n_heads * d_rope not a multiple of 8, small workspace, misaligned), ECUDA.
  */

@@ -35,12 +35,15 @@ struct GemmParams {
     void* C[2];           // [M, ldc] bf16 or fp32, row-major
     int ldc[2];           // elements
     uint64_t timeout_ns;
-    // optional epilogue work (RMSNorm split across two GEMMs): row_ss[row] += sum of
-    // the row's squared fp32 outputs; column c scaled by col_scale[c]; every row
-    // scaled by 1 / sqrt(row_ss_in[row] / rms_dim + rms_eps)
+    // optional epilogue work (RMSNorm split across two GEMMs): row_ss[t M + row] = sum
+    // of the row's squared fp32 outputs in column tile t (one column group; every
+    // (row, tile) written once, so no zeroing and no atomics); column c scaled by
+    // col_scale[c]; every row scaled by 1 / sqrt(ms / rms_dim + rms_eps), ms the sum
+    // of row_ss_in[k M + row] over k < ss_parts, in order
     float* row_ss;
     const float* col_scale;
     const float* row_ss_in;
+    int ss_parts;
     int rms_dim;
     float rms_eps;
 };
@@ -200,9 +203,12 @@ __global__ void __launch_bounds__(192, 1)
             const int row = m0 + r;
             const int N = g == 0 ? p.N[0] : p.N[1], ldc = g == 0 ? p.ldc[0] : p.ldc[1];
             void* const Cg = g == 0 ? p.C[0] : p.C[1];
-            const float rscale = p.row_ss_in != nullptr && row < p.M
-                                     ? rsqrtf(__ldg(p.row_ss_in + row) / float(p.rms_dim) + p.rms_eps)
-                                     : 1.0f;
+            float rscale = 1.0f;
+            if (p.row_ss_in != nullptr && row < p.M) {
+                float ms = 0.f;
+                for (int k = 0; k < p.ss_parts; ++k) ms += __ldg(p.row_ss_in + size_t(k) * p.M + row);
+                rscale = rsqrtf(ms / float(p.rms_dim) + p.rms_eps);
+            }
             float ss = 0.f;
 #pragma unroll 1
             for (int c = 0; c < BN; c += 32) {
@@ -247,7 +253,7 @@ __global__ void __launch_bounds__(192, 1)
                     }
                 }
             }
-            if (p.row_ss != nullptr && row < p.M) atomicAdd(p.row_ss + row, ss);
+            if (p.row_ss != nullptr && row < p.M) p.row_ss[size_t(n0 / BN) * p.M + row] = ss;
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {  // the accumulator may take tile j + 2 (rank 0's barrier counts both CTAs)

@@ -644,6 +644,7 @@ struct GemmEpilogue {
     float* row_ss = nullptr;
     const float* col_scale = nullptr;
     const float* row_ss_in = nullptr;
+    int ss_parts = 0;  // partial sums per row in row_ss_in
     int rms_dim = 1;
     float rms_eps = 0.f;
 };
@@ -689,6 +690,7 @@ int run_gemm_pair(const void* A, int M, int K, int groups, const void* B0, int N
     p.row_ss = epi.row_ss;
     p.col_scale = epi.col_scale;
     p.row_ss_in = epi.row_ss_in;
+    p.ss_parts = epi.ss_parts;
     p.rms_dim = epi.rms_dim;
     p.rms_eps = epi.rms_eps;
     const int pairs_max = max_pair_clusters(reinterpret_cast<const void*>(kern), C::THREADS, C::SMEM);
@@ -873,7 +875,9 @@ int videomla_dense_attention(const videomla_dims* dims, const void* q_nope, cons
 size_t videomla_query_projection_workspace_size(const videomla_dims* dims, int d_q, int batch, int n_tok) {
     if (!dims || d_q <= 0 || batch <= 0 || n_tok <= 0) return 0;
     const size_t m = size_t(batch) * n_tok;
-    return align256(m * 4) + m * d_q * 2;  // per-row sums of squares, then g (.) c^Q in bf16
+    // per-row partial sums of squares (one per column tile of the first GEMM, at most
+    // d_q / 128 of them), then g (.) c^Q in bf16
+    return align256(m * 4 * size_t((d_q + 127) / 128)) + m * d_q * 2;
 }
 
 int videomla_query_projection(const videomla_dims* dims, int d_q, const void* x, int batch, int n_tok,
@@ -892,18 +896,22 @@ int videomla_query_projection(const videomla_dims* dims, int d_q, const void* x,
     if (int rc = check_device()) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // RMSNorm(c^Q) = g (.) c^Q / rms(c^Q) is linear in g (.) c^Q up to the per-row factor, so it
-    // is split over the two GEMMs: the first writes g (.) c^Q (bf16) and adds each row's sum
-    // of squares of c^Q (fp32, before g and rounding); the second, both up-projections in
-    // one launch (two column groups), scales its output rows by 1 / rms.
+    // is split over the two GEMMs: the first writes g (.) c^Q (bf16) and, per column tile,
+    // each row's sum of squares of c^Q (fp32, before g and rounding); the second, both
+    // up-projections in one launch (two column groups), sums a row's parts and scales its
+    // output row by 1 / rms.
+    const int bn = gemm_pair_bn(int(M), d_q, 0, 1);
+    const int parts = (d_q + bn - 1) / bn;
     float* ss = static_cast<float*>(workspace);
-    auto* cqg = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(workspace) + align256(size_t(M) * 4));
-    if (cudaMemsetAsync(ss, 0, size_t(M) * 4, st) != cudaSuccess) return VIDEOMLA_ECUDA;
+    auto* cqg = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(workspace) +
+                                                 align256(size_t(M) * 4 * size_t((d_q + 127) / 128)));
     GemmEpilogue first;
     first.row_ss = ss;
     first.col_scale = gamma_q;
     if (int rc = gemm(x, W_dq, int(M), d_q, dims->d_model, cqg, d_q, false, st, first)) return rc;
     GemmEpilogue second;
     second.row_ss_in = ss;
+    second.ss_parts = parts;
     second.rms_dim = d_q;
     second.rms_eps = dims->rms_eps;
     return gemm2(cqg, int(M), d_q, 2, W_uq, int(nq), q_nope, int(nq), W_qr, int(nr), q_rope, int(nr), false, st,
