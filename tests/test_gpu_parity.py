@@ -303,6 +303,23 @@ def test_query_projection(dims, n_tok, B, rows, unit_gain):
     assert en <= Q_NORM_REL and er <= Q_NORM_REL
 
 
+@pytest.mark.parametrize("n_tok", [144, 4680])
+def test_query_projection_deterministic(n_tok):
+    """Each row's sum of squares is stored per column tile and added in tile
+    order, so repeated calls give bitwise-equal queries (both column-tile widths:
+    288 rows take 128-wide tiles, 4680 rows 256-wide ones)."""
+    dims = I.TINY if n_tok == 144 else I.WAN
+    B = 2 if n_tok == 144 else 1
+    pw = I.projection_weights(dims, 615, random_gamma=True)
+    x = I.tokens(dims, B, n_tok, 616).to(DEV)
+    d = _dev(pw)
+    runs = [V.query_projection(x, d["W_dq"], d["gamma_q"], d["W_uq"], d["W_qr"], dims) for _ in range(3)]
+    torch.cuda.synchronize()
+    assert V.device_status(reset=True) == V.OK
+    for qn, qr in runs[1:]:
+        assert torch.equal(qn, runs[0][0]) and torch.equal(qr, runs[0][1])
+
+
 def test_output_projection():
     dims = I.WAN
     pw = I.projection_weights(dims, 620)
