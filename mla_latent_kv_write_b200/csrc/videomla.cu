@@ -717,7 +717,8 @@ int run_gemm_pair(const void* A, int M, int K, int groups, const void* B0, int N
 }
 
 // Column tile width of the pair tiles: the one that puts the fewest columns on
-// the busiest pair of the persistent grid (ties go to 256, fewer tiles).
+// the busiest pair of the persistent grid (ties go to 256, fewer tiles).  The
+// query path counts its per-tile row sums of squares with this same choice.
 int gemm_pair_bn(int M, int N0, int N1, int groups) {
     const long long m_tiles = (M + 255) / 256;
     const int pairs = sm_count() / 2;
